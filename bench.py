@@ -1,0 +1,350 @@
+"""Benchmark of the packed variable-length attention forward on B200.
+
+Metric: effective TFLOP/s over valid FLOPs, 4 * sum(L_i^2) * d * H per call
+(block-diagonal work only; masked tail work and padding do not count), on the
+mixed-resolution pack (512x512, 1024x1024 and 768x432 images at patch 16 ->
+segments [1024, 4096, 1296], 24 heads, head_dim 128, bf16).  One step = one
+call of the C-ABI entry point ``pa_varlen_attn_fwd`` (schedule kernel +
+attention kernel) on inputs resident in HBM; L2 is flushed between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own pack of the same
+shape (independent replicas: the forward has no exchange step), the timed
+region is bracketed by barriers, and the time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on bounded samples of the same
+workload on the host cores.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(x, world, device):
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if not self.rows:
+            return None
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def workload_desc(cfg):
+    segs = cfg["segments"]
+    desc = {"workload": f"{cfg['name']} pack: {cfg.get('description', '')}",
+            "segments": segs if len(segs) <= 32 else f"{len(segs)} segments",
+            "total_tokens": int(sum(segs)), "heads": cfg["heads"], "head_dim": cfg["head_dim"],
+            "valid_flops_per_step": workloads.valid_flops(segs, cfg["heads"], cfg["head_dim"])}
+    return desc
+
+
+def oracle_sample_rate(p, cfg, target_s, seed=0, max_rows=None):
+    """Times the fp64 oracle on a bounded random sample of (token, head) rows; returns
+    (TFLOP/s over the sample's valid FLOPs, rows, seconds, threads)."""
+    import oracle
+    segs = cfg["segments"]
+    T, H, d = sum(segs), cfg["heads"], cfg["head_dim"]
+    cu = np.concatenate([[0], np.cumsum(segs)])
+    seg_len = np.repeat(np.array(segs), segs)  # length of the segment of every token
+    rng = np.random.default_rng(seed)
+    n = 8
+    while True:
+        tok = rng.integers(0, T, size=n)
+        head = rng.integers(0, H, size=n).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.varlen_attention(p["q"], p["k"], p["v"], cu, p["scale"], rows=(tok, head))
+        dt = time.perf_counter() - t0
+        if dt >= target_s or (max_rows and n >= max_rows):
+            flops = float(np.sum(4.0 * seg_len[tok] * d))
+            return flops / dt / 1e12, n, dt, oracle.default_threads()
+        n = int(n * min(8.0, max(2.0, 1.2 * target_s / max(dt, 1e-4))))
+        if max_rows:
+            n = min(n, max_rows)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    cfg = workloads.load_config(args.config)
+    p = workloads.make_inputs(cfg)
+    # size one step so that (warmup + steps) samples take about two minutes in all
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    rates = []
+    rows = secs = threads = 0
+    for i in range(args.warmup + args.steps):
+        r, rows, secs, threads = oracle_sample_rate(p, cfg, per_step, seed=i)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.median(rates)
+    flops = workloads.valid_flops(cfg["segments"], cfg["heads"], cfg["head_dim"])
+    line = {"impl": "reference", "metric": BASELINE_METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": flops / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(workload_desc(cfg), parallelism="host cores"),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{rows} random (token, head) rows per step, about {secs:.1f} s each; "
+                                       "rate extrapolated to the whole pack by valid FLOPs"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+BASELINE_METRIC = "varlen attn fwd effective TFLOP/s (valid FLOPs) on 1 B200; % of BF16 peak"
+
+
+def traffic_for_current_kernel():
+    """DRAM bytes per launch from the committed ncu summary, if it matches the kernel source as built."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("sources_sha256"):
+        return None
+    return rec
+
+
+def run_ours(args, world, rank, local):
+    import dit_resolution_packed_b200 as pa
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = workloads.load_config(args.config)
+    cfg_r = dict(cfg, seed=int(cfg["seed"]) + 7919 * rank)  # each replica its own data, same shapes
+    p = workloads.make_inputs(cfg_r)
+    segs = cfg["segments"]
+    T, H, d = sum(segs), cfg["heads"], cfg["head_dim"]
+    flops = workloads.valid_flops(segs, H, d)
+    q, k, v = (p[n].to(device) for n in ("q", "k", "v"))
+    cu = p["cu_seqlens"].to(device)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, H, dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        rc = pa.pa_varlen_attn_fwd(q, k, v, cu, p["max_seqlen"], p["scale"], out, lse, stream)
+        if rc != pa.PA_OK:
+            raise pa.PackAttnError(rc, "pa_varlen_attn_fwd")
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, "warm-up")
+
+    # ---- device-resident timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    pa.pa_profile_read()  # clear
+    pa.pa_profile_enable(True)
+    for i in range(args.steps):
+        flush.fill_(1.0)  # evict q/k/v/out from L2 between steps (untimed)
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    pa.pa_profile_enable(False)
+    barrier(world)
+    clock_rec = clocks.stop() if clocks else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_ms_total, kern_n = pa.pa_profile_read()
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, "timed region")
+    total_ms = allreduce_max(sum(step_ms), world, device)
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    hq, hk, hv = (p[n].pin_memory() for n in ("q", "k", "v"))
+    hcu = p["cu_seqlens"].pin_memory()
+    hout = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    hlse = torch.empty(T, H, dtype=torch.float32).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+
+    def e2e_step(i=None):
+        if i is not None:
+            e2e_ev[i][0].record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        cu.copy_(hcu, non_blocking=True)
+        call()
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+        if i is not None:
+            e2e_ev[i][1].record(stream)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.fill_(1.0)
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = allreduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev), world, device) / args.steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    kern_avg_s = kern_ms_total / max(1, kern_n) * 1e-3
+    achieved = flops / kern_avg_s / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    trec = traffic_for_current_kernel()
+    line = {
+        "metric": BASELINE_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_desc(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
+                       parallelism=f"{world} independent replica(s), no collective"),
+        "pct_of_bf16_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"bf16_tflops ({peak_src}, burst)",
+                     "kernel": "attn_fwd_kernel<128>" if d == 128 else "attn_fwd_kernel<64>",
+                     "traffic": (trec or {}).get("dram_bytes_per_launch")},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clock_rec,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        r, rows, secs, threads = oracle_sample_rate(p, cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": r, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{rows} random (token, head) rows of the same pack, {secs:.1f} s; "
+                                          "rate = valid FLOPs of those rows / wall time"}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", default="mixed", choices=workloads.CONFIG_NAMES)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+"""B200 (sm_100a) packed variable-length attention: Python binding of ``libpackattn.so``.
+
+The functions named ``pa_*`` mirror the C ABI in ``include/packattn.h`` one to
+one and only marshal arguments (torch tensors -> device pointers, the current
+CUDA stream -> ``cudaStream_t``).  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback: if the library is
+missing or cannot be loaded, every call raises.
+
+``varlen_attn_fwd`` is the convenience form: it allocates ``out`` and ``lse``,
+calls ``pa_varlen_attn_fwd`` and raises on a host-side error status.
+"""
+import ctypes
+import math
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpackattn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "packattn.h")
+
+PA_OK = 0
+PA_ERR_NULL = -1
+PA_ERR_ALIGN = -2
+PA_ERR_HEAD_DIM = -3
+PA_ERR_SHAPE = -4
+PA_ERR_CU_SEQLENS = -5
+PA_ERR_MAX_SEQLEN = -6
+PA_ERR_TIMEOUT = -7
+PA_ERR_CUDA = -8
+PA_ERR_SCALE = -9
+PA_ERR_NOT_DEVICE = -10
+
+_lib = None
+
+
+class PackAttnError(RuntimeError):
+    def __init__(self, code, where=""):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})" if where else status_string(code))
+
+
+def load_library(path=None):
+    """Loads the in-tree C-ABI library (built by ``_build.py`` / ``__graft_entry__.build()``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m dit_resolution_packed_b200._build` "
+                           "(there is no fallback implementation)")
+    lib = ctypes.CDLL(p)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.pa_varlen_attn_fwd.restype = ctypes.c_int
+    lib.pa_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp]
+    lib.pa_get_error.restype = ctypes.c_int
+    lib.pa_get_error.argtypes = [vp]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_status_string.argtypes = [ctypes.c_int]
+    lib.pa_version.restype = ctypes.c_int
+    lib.pa_version.argtypes = []
+    lib.pa_release_workspace.restype = None
+    lib.pa_release_workspace.argtypes = []
+    lib.pa_set_wait_limit_ms.restype = None
+    lib.pa_set_wait_limit_ms.argtypes = [ctypes.c_int]
+    lib.pa_selftest_wait_timeout.restype = ctypes.c_int
+    lib.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+    lib.pa_profile_enable.restype = None
+    lib.pa_profile_enable.argtypes = [ctypes.c_int]
+    lib.pa_profile_read.restype = ctypes.c_int
+    lib.pa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int32)]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def header_functions(path=HEADER_PATH):
+    """Names of the functions ``include/packattn.h`` declares."""
+    with open(path) as f:
+        text = f.read()
+    return re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def pa_varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale, out, lse, stream=None):
+    """C ``pa_varlen_attn_fwd`` on torch tensors: q, k, v, out bf16 [T, H, d]; cu_seqlens int32 [B+1];
+    lse fp32 [T, H].  Returns the status code (enqueued on ``stream``, default: the current stream)."""
+    import torch
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("out", out, torch.bfloat16), ("cu_seqlens", cu_seqlens, torch.int32),
+                        ("lse", lse, torch.float32)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    T, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or out.shape != q.shape or tuple(lse.shape) != (T, H):
+        raise ValueError("shape mismatch: q, k, v, out [T, H, d]; lse [T, H]")
+    B = cu_seqlens.numel() - 1
+    return load_library().pa_varlen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, T, H, d,
+                                             int(max_seqlen), float(scale), _ptr(out), _ptr(lse),
+                                             _stream_handle(stream))
+
+
+def varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale=None, out=None, lse=None, stream=None):
+    """Packed varlen bidirectional attention forward; returns (out bf16 [T, H, d], lse fp32 [T, H])."""
+    import torch
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    rc = pa_varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale, out, lse, stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_varlen_attn_fwd")
+    return out, lse
+
+
+def pa_get_error(stream=None):
+    return load_library().pa_get_error(_stream_handle(stream))
+
+
+def pa_status_string(code):
+    return load_library().pa_status_string(int(code)).decode()
+
+
+status_string = pa_status_string
+
+
+def pa_version():
+    return load_library().pa_version()
+
+
+def pa_release_workspace():
+    load_library().pa_release_workspace()
+
+
+def pa_set_wait_limit_ms(ms):
+    load_library().pa_set_wait_limit_ms(int(ms))
+
+
+def pa_selftest_wait_timeout(limit_us, stream=None):
+    return load_library().pa_selftest_wait_timeout(int(limit_us), _stream_handle(stream))
+
+
+def pa_profile_enable(on):
+    load_library().pa_profile_enable(1 if on else 0)
+
+
+def pa_profile_read():
+    """(summed attention-kernel milliseconds, launches) since the last read."""
+    ms, n = ctypes.c_double(0.0), ctypes.c_int32(0)
+    rc = load_library().pa_profile_read(ctypes.byref(ms), ctypes.byref(n))
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_profile_read")
+    return ms.value, n.value

@@ -1,0 +1,521 @@
+// attn_fwd_sm100.cuh -- packed variable-length bidirectional attention forward
+// for B200 (sm_100a): TMA tile loads, tcgen05 MMAs accumulating in tensor
+// memory, online softmax in registers, TMA stores of the output.
+//
+// Math (SparseAttn page, section 3.1; GigaPath-Flash page, sections 3.2/4.2 for
+// the blockwise online softmax): per query row, with x = scale*log2(e)*q.k,
+//     m  = running max used for the exponentials,
+//     P  = exp2(x - m),  l = l*exp2(m_old - m) + rowsum(P),
+//     O  = O*exp2(m_old - m) + P V,
+//     out = O / l,   lse = (m + log2 l) * ln 2.
+// The exponent shift m is only moved when a new tile's max exceeds it by more
+// than kRescaleLog2 (then O and l are rescaled); otherwise P <= 2^kRescaleLog2
+// and the result is unchanged, because out and lse do not depend on m.
+//
+// Work item = (segment, head, pair of 128-row query tiles).  CTA layout, 12 warps:
+//   warps 0-3  softmax + epilogue of query tile 0 (one thread per row)
+//   warps 4-7  softmax + epilogue of query tile 1
+//   warp 8     TMA producer: Q tiles, then K_j, V_j into a ring of smem slots
+//   warp 9     tensor-memory owner and MMA issuer
+//   warps 10-11 idle (they complete the third warpgroup for the register split)
+// Tensor memory (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1.  P (bf16)
+// overwrites the first half of its S columns and feeds the P.V MMA from tensor
+// memory.  Ping-pong: while warps 0-3 turn S0 into P0, the tensor core runs
+// S1 = Q1 K^T, and the other way round.
+#pragma once
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace pa {
+
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kFwdThreads = 384;
+// Register split of the 384-thread block launched at 168 registers per thread
+// (384 x 168 = 64512): the two softmax warpgroups rise to 192, the producer /
+// MMA warpgroup drops to 120.  2*128*192 + 128*120 = 64512.  The build checks
+// that the kernels are compiled at exactly kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 192;
+constexpr int kControlRegs = 120;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kFwdThreads * kLaunchRegs, "register split");
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int kRows = 128;                      // rows of a Q/K/V/O tile
+  static constexpr int kTileBytes = kRows * D * 2;       // bf16 tile
+  static constexpr int kColBlocks = D / 64;              // 128-byte swizzle atoms across d
+  static constexpr int kBlockBytes = kRows * 128;        // one 64-column block of a tile
+  static constexpr int kSlots = (D == 128) ? 3 : 6;      // K/V ring depth
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffO = kOffKV + kSlots * kTileBytes;
+  static constexpr int kOffBar = kOffO + 2 * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // + 1024 for base alignment
+  static constexpr uint32_t kTmemCols = 512;
+  __host__ __device__ static constexpr uint32_t col_s(int tile) { return tile ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t col_o(int tile) { return tile ? 256u + D : 256u; }
+};
+
+struct FwdParams {
+  const int32_t* cu;
+  float* lse;
+  const int32_t* counts;      // [0] items, [1] ordered segments
+  const int32_t* order;
+  const int32_t* item_start;
+  const uint8_t* maps;        // [B][4] tensor maps: q, k, v, out
+  int32_t* status;
+  int32_t heads;
+  float scale_log2;           // scale * log2(e)
+  uint64_t wait_limit_ns;
+  int32_t err_timeout;
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[8], kv_empty[8];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t epi_free[2], epi_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct WorkItem {
+  int32_t seg, beg, len, head, q0, nkv;
+  bool two;  // second query tile has rows
+};
+
+__device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p, int32_t n_sorted) {
+  int32_t lo = 0, hi = n_sorted;
+  while (hi - lo > 1) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (__ldg(p.item_start + mid) <= item) lo = mid; else hi = mid;
+  }
+  WorkItem w;
+  w.seg = __ldg(p.order + lo);
+  const int32_t local = item - __ldg(p.item_start + lo);
+  w.beg = __ldg(p.cu + w.seg);
+  w.len = __ldg(p.cu + w.seg + 1) - w.beg;
+  const int32_t npairs = (w.len + 255) >> 8;
+  w.head = local / npairs;
+  w.q0 = (local - w.head * npairs) * 256;
+  w.nkv = (w.len + 127) >> 7;
+  w.two = w.q0 + 128 < w.len;
+  return w;
+}
+
+__device__ __forceinline__ const void* seg_map(const FwdParams& p, int32_t seg, int which) {
+  return p.maps + (static_cast<size_t>(seg) * 4 + which) * 128;
+}
+
+// A wait used while draining after an abort: ignores the abort flag, bounded by its own limit.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ producer
+template <int D>
+__device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, Bars* bars, const WaitCtl& wc,
+                                             int32_t n_items, int32_t n_sorted) {
+  using C = FwdCfg<D>;
+  int slot = 0;
+  uint32_t phase = 0;
+  uint32_t q_round = 0;
+  // last armed phase of every slot, for the drain after an abort
+  uint32_t armed = 0, armed_phase = 0;
+  bool q_armed = false;
+  uint32_t q_armed_phase = 0;
+  bool ok = true;
+  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    const WorkItem w = decode_item(item, p, n_sorted);
+    const void* mq = seg_map(p, w.seg, 0);
+    const void* mk = seg_map(p, w.seg, 1);
+    const void* mv = seg_map(p, w.seg, 2);
+    fence_tmap_acquire(mq);
+    fence_tmap_acquire(mk);
+    fence_tmap_acquire(mv);
+    const int32_t xcol = w.head * D;
+    if (!(ok = mbar_wait(&bars->q_empty, (q_round & 1u) ^ 1u, wc))) break;
+    mbar_arrive_expect_tx(&bars->q_full, (w.two ? 2u : 1u) * C::kTileBytes);
+    q_armed = true;
+    q_armed_phase = q_round & 1u;
+#pragma unroll
+    for (int cb = 0; cb < C::kColBlocks; ++cb) {
+      tma_load_2d(smem + C::kOffQ + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0, &bars->q_full);
+      if (w.two)
+        tma_load_2d(smem + C::kOffQ + C::kTileBytes + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0 + 128,
+                    &bars->q_full);
+    }
+    ++q_round;
+    for (int32_t j = 0; ok && j < w.nkv; ++j) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        if (!(ok = mbar_wait(&bars->kv_empty[slot], phase ^ 1u, wc))) break;
+        mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
+        armed |= 1u << slot;
+        armed_phase = (armed_phase & ~(1u << slot)) | (phase << slot);
+        uint8_t* dst = smem + C::kOffKV + slot * C::kTileBytes;
+        const void* m = which ? mv : mk;
+#pragma unroll
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, j * 128, &bars->kv_full[slot]);
+        if (++slot == C::kSlots) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Let every copy this thread started land before the CTA can exit.
+    const uint64_t lim = wc.limit_ns;
+    for (int s = 0; s < C::kSlots; ++s)
+      if (armed & (1u << s)) drain_wait(&bars->kv_full[s], (armed_phase >> s) & 1u, lim);
+    if (q_armed) drain_wait(&bars->q_full, q_armed_phase, lim);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * FwdCfg<D>::kBlockBytes + (kk & 3) * 32;
+    mma_bf16_ss(d_tmem, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc,
+                kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    mma_bf16_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_addr + kk * 16 * 128, FwdCfg<D>::kBlockBytes, 1024), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, const WaitCtl& wc,
+                                        uint32_t tmem, int32_t n_items, int32_t n_sorted) {
+  using C = FwdCfg<D>;
+  const uint32_t q_addr0 = smem_u32(smem + C::kOffQ);
+  const uint32_t kv_addr0 = smem_u32(smem + C::kOffKV);
+  int slot = 0;
+  uint32_t phase = 0, q_round = 0;
+  uint32_t p_ph = 0, oe_ph = 0;  // bit t: phase of tile t
+  bool ok = true;
+  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    const WorkItem w = decode_item(item, p, n_sorted);
+    if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
+    ++q_round;
+    int ks = slot;
+    if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
+    if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
+    tc_fence_after();
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (t == 1 && !w.two) break;
+      issue_s<D>(tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
+      mma_commit(&bars->s_full[t]);
+    }
+    mma_commit(&bars->kv_empty[ks]);
+    if (w.nkv == 1) mma_commit(&bars->q_empty);
+    for (int32_t j = 0; ok && j < w.nkv; ++j) {
+      const bool has_next = j + 1 < w.nkv;
+      const int vs = slot;
+      if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
+      if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
+      if (has_next) {
+        ks = slot;
+        if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
+        if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
+      }
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t == 1 && !w.two) break;
+        if (j == 0) {
+          if (!(ok = mbar_wait(&bars->o_empty[t], ((oe_ph >> t) & 1u) ^ 1u, wc))) break;
+          oe_ph ^= 1u << t;
+        }
+        if (!(ok = mbar_wait(&bars->p_full[t], (p_ph >> t) & 1u, wc))) break;
+        p_ph ^= 1u << t;
+        tc_fence_after();
+        issue_pv<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, j > 0);
+        if (has_next) {
+          issue_s<D>(tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
+          mma_commit(&bars->s_full[t]);
+        } else {
+          mma_commit(&bars->o_full[t]);
+        }
+      }
+      if (!ok) break;
+      mma_commit(&bars->kv_empty[vs]);
+      if (has_next) {
+        mma_commit(&bars->kv_empty[ks]);
+        if (j + 2 == w.nkv) mma_commit(&bars->q_empty);
+      }
+    }
+  }
+  // Every MMA issued so far completes before tensor memory is released.
+  mma_commit(&bars->drain);
+  drain_wait(&bars->drain, 0, wc.limit_ns);
+}
+
+// ------------------------------------------------------------------ softmax + epilogue
+template <int D>
+__device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, Bars* bars, const WaitCtl& wc,
+                                            uint32_t tmem, int32_t n_items, int32_t n_sorted, int tile) {
+  using C = FwdCfg<D>;
+  const int t = threadIdx.x & 127;  // row of the query tile
+  const int lane = threadIdx.x & 31;
+  const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
+  const uint32_t tS = tmem + lane_base + C::col_s(tile);
+  const uint32_t tO = tmem + lane_base + C::col_o(tile);
+  uint8_t* stage = smem + C::kOffO + tile * C::kTileBytes;
+  const float c = p.scale_log2;
+  uint32_t s_ph = 0, of_ph = 0, ef_ph = 0, eful_ph = 0;
+  bool ok = true;
+
+  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    const WorkItem w = decode_item(item, p, n_sorted);
+    if (tile == 1 && !w.two) continue;
+    // l: sum of the fp32 exponentials (gives lse); lr: sum of the same values rounded to
+    // bf16, i.e. of the weights the P.V product actually used (normalises the output,
+    // so each output row is an exact convex combination of value rows).
+    float m = 0.f, l = 0.f, lr = 0.f;
+    for (int32_t j = 0; j < w.nkv; ++j) {
+      ok = mbar_wait(&bars->s_full[tile], s_ph, wc);
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      s_ph ^= 1u;
+      tc_fence_after();
+      uint32_t r[128];
+      PA_TMEM_LD32(tS + 0, (r + 0));
+      PA_TMEM_LD32(tS + 32, (r + 32));
+      PA_TMEM_LD32(tS + 64, (r + 64));
+      PA_TMEM_LD32(tS + 96, (r + 96));
+      tmem_wait_ld();
+      const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment (masked above)
+      const bool partial = kv_valid < 128;
+      float mx;
+      if (c >= 0.f) {
+        mx = -INFINITY;
+        if (!partial) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mx = fmaxf(mx, k < kv_valid ? __uint_as_float(r[k]) : -INFINITY);
+        }
+      } else {
+        mx = INFINITY;
+        if (!partial) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mx = fminf(mx, __uint_as_float(r[k]));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 128; ++k) mx = fminf(mx, k < kv_valid ? __uint_as_float(r[k]) : INFINITY);
+        }
+      }
+      const float xmax = mx * c;  // largest scaled score of the row in this tile (log2 units)
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m = xmax;
+      } else if (__any_sync(0xffffffffu, xmax > m + kRescaleLog2)) {
+        const float m_new = fmaxf(m, xmax);
+        alpha = ex2_approx(m - m_new);
+        l *= alpha;
+        lr *= alpha;
+        m = m_new;
+        rescale = true;
+      }
+      const float neg_m = -m;
+      float rs = 0.f, rsr = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int k0 = cc * 32 + 2 * k;
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[k0]), c, neg_m));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[k0 + 1]), c, neg_m));
+          if (partial) {
+            p0 = k0 < kv_valid ? p0 : 0.f;
+            p1 = k0 + 1 < kv_valid ? p1 : 0.f;
+          }
+          const uint32_t pr = pack_bf16x2(p0, p1);
+          rs += p0 + p1;
+          rsr += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
+          pk[k] = pr;
+        }
+        PA_TMEM_ST16(tS + cc * 16, pk);
+      }
+      if (rescale) {
+        // O += P V of the previous tile has completed (S of this tile was issued after it).
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          PA_TMEM_LD32(tO + cc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          PA_TMEM_ST32(tO + cc * 32, o);
+        }
+      }
+      l += rs;
+      lr += rsr;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[tile]);
+    }
+    if (!ok) break;
+
+    // ---- epilogue: O / l -> bf16 -> swizzled staging tile -> TMA store (clipped at the segment end)
+    ok = mbar_wait(&bars->o_full[tile], of_ph, wc);
+    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+    of_ph ^= 1u;
+    tc_fence_after();
+    if (t == 0) {
+      bulk_wait_group_read0();  // the previous store has finished reading the staging tile
+      mbar_arrive(&bars->epi_free[tile]);
+    }
+    ok = mbar_wait(&bars->epi_free[tile], ef_ph, wc);
+    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+    ef_ph ^= 1u;
+    const float inv_l = 1.0f / lr;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      PA_TMEM_LD32(tO + cc * 32, o);
+      tmem_wait_ld();
+      uint8_t* row = stage + (cc >> 1) * C::kBlockBytes + t * 128;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 v;
+        v.x = pack_bf16x2(__uint_as_float(o[q4 * 8 + 0]) * inv_l, __uint_as_float(o[q4 * 8 + 1]) * inv_l);
+        v.y = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2]) * inv_l, __uint_as_float(o[q4 * 8 + 3]) * inv_l);
+        v.z = pack_bf16x2(__uint_as_float(o[q4 * 8 + 4]) * inv_l, __uint_as_float(o[q4 * 8 + 5]) * inv_l);
+        v.w = pack_bf16x2(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
+        const int chunk = (cc & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
+        *reinterpret_cast<uint4*>(row + ((chunk ^ (t & 7)) << 4)) = v;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->o_empty[tile]);  // O columns may be overwritten now
+    fence_proxy_async_smem();
+    mbar_arrive(&bars->epi_full[tile]);
+    const int32_t row0 = w.q0 + tile * 128;
+    if (t == 0) {
+      // A failed wait here only skips the store; the abort flag stops every role at its next wait.
+      if (mbar_wait(&bars->epi_full[tile], eful_ph, wc)) {
+        const void* mo = seg_map(p, w.seg, 3);
+        fence_tmap_acquire(mo);
+#pragma unroll
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_store_2d(mo, w.head * D + cb * 64, row0, stage + cb * C::kBlockBytes);
+        bulk_commit_group();
+      }
+    }
+    eful_ph ^= 1u;
+    if (row0 + t < w.len) {
+      const float lse2 = m + __log2f(l);
+      p.lse[static_cast<size_t>(w.beg + row0 + t) * p.heads + w.head] = lse2 * 0.69314718055994531f;
+    }
+  }
+  if (t == 0) bulk_wait_group0();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
+  const int warp = threadIdx.x >> 5;
+  const int32_t n_items = p.counts[0];
+  const int32_t n_sorted = p.counts[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 4);
+      mbar_init(&bars->o_full[t], 1);
+      mbar_init(&bars->o_empty[t], 4);
+      mbar_init(&bars->epi_free[t], 1);
+      mbar_init(&bars->epi_full[t], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtl wc{&bars->abort_flag, p.status, p.wait_limit_ns, p.err_timeout};
+
+  // The two register regions never merge again: each branch ends with its own
+  // barrier over the whole block, and only the tensor-memory owner continues.
+  if (warp < 8) {
+    regs_increase<kSoftmaxRegs>();
+    run_softmax<D>(p, smem, bars, wc, tmem, n_items, n_sorted, warp >> 2);
+    tc_fence_before();
+    named_bar_sync(1, kFwdThreads);
+  } else {
+    regs_decrease<kControlRegs>();
+    if (warp == 8) {
+      if ((threadIdx.x & 31) == 0) run_producer<D>(p, smem, bars, wc, n_items, n_sorted);
+    } else if (warp == 9) {
+      if ((threadIdx.x & 31) == 0) run_mma<D>(p, smem, bars, wc, tmem, n_items, n_sorted);
+    }
+    __syncwarp();
+    tc_fence_before();
+    named_bar_sync(1, kFwdThreads);
+    if (warp == 9) {
+      tc_fence_after();
+      tmem_dealloc(tmem, C::kTmemCols);
+    }
+  }
+}
+
+// A one-warp kernel that waits on a barrier nothing completes, through the same
+// bounded wait as the attention kernel; it must record a timeout and return.
+__global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns, int32_t err_timeout) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl wc{&abort_flag, status, limit_ns, err_timeout};
+  mbar_wait(&bar, 0, wc);
+  __syncthreads();
+}
+
+}  // namespace pa

@@ -1,0 +1,343 @@
+// packattn.cu -- host side of the C ABI declared in include/packattn.h.
+//
+// A call validates its arguments on the host, finds (or grows) the workspace of
+// its (device, stream) pair, encodes four template tensor maps over the whole
+// q / k / v / out matrices, and enqueues two kernels on the caller's stream:
+// the segment scheduler (one CTA) and the persistent attention kernel (one CTA
+// per SM).  Nothing synchronises on this path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attn_fwd_sm100.cuh"
+#include "packattn.h"
+#include "schedule.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+};
+
+struct StreamState {
+  int device = -1;
+  cudaStream_t stream = nullptr;
+  int32_t* status = nullptr;  // never moves once allocated
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+std::vector<StreamState*> g_states;
+DeviceInfo g_dev[64];
+int g_wait_limit_ms = 4000;
+
+// profiling
+bool g_prof_on = false;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_events;
+size_t g_prof_used = 0;
+
+constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t counts, order, item_start, maps, total;
+};
+
+WsLayout ws_layout(int32_t batch) {
+  WsLayout L;
+  L.counts = 0;
+  L.order = 128;
+  L.item_start = align_up(L.order + 4 * static_cast<size_t>(batch), 128);
+  L.maps = align_up(L.item_start + 4 * (static_cast<size_t>(batch) + 1), 128);
+  L.total = L.maps + 512 * static_cast<size_t>(batch);
+  return L;
+}
+
+int device_of(const void* ptr, int* dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_NOT_DEVICE;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return PA_ERR_NOT_DEVICE;
+  *dev = a.device;
+  return PA_OK;
+}
+
+// Finds or creates the state of (device, stream); the device must be current.  g_mu held.
+StreamState* state_for(int device, cudaStream_t stream) {
+  for (StreamState* s : g_states)
+    if (s->device == device && s->stream == stream) return s;
+  StreamState* s = new StreamState();
+  s->device = device;
+  s->stream = stream;
+  g_states.push_back(s);
+  return s;
+}
+
+int ensure_status(StreamState* s) {
+  if (s->status) return PA_OK;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&s->status), 128, s->stream) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemsetAsync(s->status, 0, 128, s->stream) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+int ensure_workspace(StreamState* s, size_t bytes) {
+  if (s->ws_bytes >= bytes) return PA_OK;
+  if (s->ws) cudaFreeAsync(s->ws, s->stream);
+  s->ws = nullptr;
+  s->ws_bytes = 0;
+  const size_t want = std::max<size_t>(bytes + bytes / 2, 64 * 1024);
+  if (cudaMallocAsync(reinterpret_cast<void**>(&s->ws), want, s->stream) != cudaSuccess) return PA_ERR_CUDA;
+  s->ws_bytes = want;
+  return PA_OK;
+}
+
+int ensure_device(int device) {
+  if (device < 0 || device >= 64) return PA_ERR_CUDA;
+  DeviceInfo& d = g_dev[device];
+  if (d.ready) return PA_OK;
+  if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::FwdCfg<64>::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::FwdCfg<128>::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  d.ready = true;
+  return PA_OK;
+}
+
+bool encode_map(CUtensorMap* m, const void* base, int32_t rows, int32_t heads, int32_t head_dim) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(heads) * head_dim, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(heads) * head_dim * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                       int32_t total_tokens, int32_t heads, int32_t head_dim, int32_t max_seqlen, float scale,
+                       void* out, float* lse, void* stream_handle) {
+  // ---- host-visible argument checks: nothing is enqueued on failure
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SCALE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  if (max_seqlen < 1) return PA_ERR_MAX_SEQLEN;
+  if (!q || !k || !v || !cu_seqlens || !out || !lse) return PA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+      !aligned(cu_seqlens, 4))
+    return PA_ERR_ALIGN;
+  // work items: heads * sum ceil(L_i / 256) <= heads * (ceil(T / 256) + batch) must fit int32
+  const int64_t item_bound = static_cast<int64_t>(heads) * ((static_cast<int64_t>(total_tokens) + 255) / 256 + batch);
+  if (item_bound >= (int64_t(1) << 31) || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24))
+    return PA_ERR_SHAPE;
+
+  int dev = -1, d2 = -1;
+  int rc;
+  if ((rc = device_of(q, &dev)) != PA_OK) return rc;
+  const void* others[5] = {k, v, out, lse, cu_seqlens};
+  for (const void* p : others) {
+    if ((rc = device_of(p, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  const WsLayout L = ws_layout(batch);
+  if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
+
+  pa::SchedParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  const void* bases[4] = {q, k, v, out};
+  for (int i = 0; i < 4; ++i) {
+    if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
+    sp.base[i] = bases[i];
+  }
+  sp.cu = cu_seqlens;
+  sp.status = st->status;
+  sp.counts = reinterpret_cast<int32_t*>(st->ws + L.counts);
+  sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
+  sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
+  sp.maps = st->ws + L.maps;
+  sp.row_bytes = static_cast<uint64_t>(heads) * head_dim * 2;
+  sp.batch = batch;
+  sp.total = total_tokens;
+  sp.heads = heads;
+  sp.max_seqlen = max_seqlen;
+  sp.err_cu = PA_ERR_CU_SEQLENS;
+  sp.err_max = PA_ERR_MAX_SEQLEN;
+  pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  pa::FwdParams fp;
+  fp.cu = cu_seqlens;
+  fp.lse = lse;
+  fp.counts = sp.counts;
+  fp.order = sp.order;
+  fp.item_start = sp.item_start;
+  fp.maps = sp.maps;
+  fp.status = st->status;
+  fp.heads = heads;
+  fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  fp.err_timeout = PA_ERR_TIMEOUT;
+  const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
+
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (g_prof_on) {
+    if (g_prof_used == g_prof_events.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return PA_ERR_CUDA;
+      g_prof_events.emplace_back(a, b);
+    }
+    ev0 = g_prof_events[g_prof_used].first;
+    ev1 = g_prof_events[g_prof_used].second;
+    ++g_prof_used;
+    cudaEventRecord(ev0, stream);
+  }
+  if (head_dim == 128)
+    pa::attn_fwd_kernel<128><<<grid, pa::kFwdThreads, pa::FwdCfg<128>::kSmemBytes, stream>>>(fp);
+  else
+    pa::attn_fwd_kernel<64><<<grid, pa::kFwdThreads, pa::FwdCfg<64>::kSmemBytes, stream>>>(fp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (g_prof_on) cudaEventRecord(ev1, stream);
+  return PA_OK;
+}
+
+int pa_get_error(void* stream_handle) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (stream != nullptr) {
+    if (cudaStreamGetDevice(stream, &dev) != cudaSuccess) return PA_ERR_CUDA;
+  } else if (cudaGetDevice(&dev) != cudaSuccess) {
+    return PA_ERR_CUDA;
+  }
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+  StreamState* st = nullptr;
+  for (StreamState* s : g_states)
+    if (s->device == dev && s->stream == stream) st = s;
+  if (!st || !st->status) return PA_OK;
+  int32_t h = 0;
+  if (cudaMemcpy(&h, st->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return PA_ERR_CUDA;
+  if (h != 0 && cudaMemset(st->status, 0, 4) != cudaSuccess) return PA_ERR_CUDA;
+  return h;
+}
+
+const char* pa_status_string(int code) {
+  switch (code) {
+    case PA_OK: return "ok";
+    case PA_ERR_NULL: return "a required pointer is NULL";
+    case PA_ERR_ALIGN: return "pointer misaligned (q/k/v/out need 16 bytes, lse/cu_seqlens 4 bytes)";
+    case PA_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
+    case PA_ERR_SHAPE: return "invalid sizes (heads, batch, total_tokens)";
+    case PA_ERR_CU_SEQLENS: return "invalid cu_seqlens (must start at 0, not decrease, end at total_tokens)";
+    case PA_ERR_MAX_SEQLEN: return "max_seqlen below 1 or below a segment length";
+    case PA_ERR_TIMEOUT: return "a device pipeline wait exceeded its limit";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_SCALE: return "scale is not finite";
+    case PA_ERR_NOT_DEVICE: return "a buffer is not device memory of one GPU";
+    default: return "unknown status";
+  }
+}
+
+int pa_version(void) { return 100; }
+
+void pa_release_workspace(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (StreamState* s : g_states) {
+    if (cudaSetDevice(s->device) == cudaSuccess) {
+      cudaDeviceSynchronize();
+      if (s->ws) cudaFree(s->ws);
+      if (s->status) cudaFree(s->status);
+    }
+    delete s;
+  }
+  g_states.clear();
+}
+
+void pa_set_wait_limit_ms(int ms) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_wait_limit_ms = ms < 1 ? 1 : ms;
+}
+
+int pa_selftest_wait_timeout(uint32_t limit_us, void* stream_handle) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (stream != nullptr) {
+    if (cudaStreamGetDevice(stream, &dev) != cudaSuccess) return PA_ERR_CUDA;
+  } else if (cudaGetDevice(&dev) != cudaSuccess) {
+    return PA_ERR_CUDA;
+  }
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  StreamState* st = state_for(dev, stream);
+  if (ensure_status(st) != PA_OK) return PA_ERR_CUDA;
+  pa::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(st->status, static_cast<uint64_t>(limit_us) * 1000ull,
+                                                         PA_ERR_TIMEOUT);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+void pa_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_prof_on = on != 0;
+}
+
+int pa_profile_read(double* total_ms, int32_t* launches) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  double sum = 0.0;
+  for (size_t i = 0; i < g_prof_used; ++i) {
+    if (cudaEventSynchronize(g_prof_events[i].second) != cudaSuccess) return PA_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof_events[i].first, g_prof_events[i].second) != cudaSuccess) return PA_ERR_CUDA;
+    sum += ms;
+  }
+  if (total_ms) *total_ms = sum;
+  if (launches) *launches = static_cast<int32_t>(g_prof_used);
+  g_prof_used = 0;
+  return PA_OK;
+}
+
+}  // extern "C"

