@@ -12,7 +12,10 @@
 // than kRescaleLog2 (then O and l are rescaled); otherwise P <= 2^kRescaleLog2
 // and the result is unchanged, because out and lse do not depend on m.
 //
-// Work item = (segment, head, pair of 128-row query tiles).  CTA layout, 12 warps:
+// Work item = (segment, head, pair of 128-row query tiles).  Items are taken
+// longest first from a global counter by the producer warp (dynamic
+// longest-processing-time scheduling) and handed to the other warps through a
+// two-slot shared-memory ring.  CTA layout, 12 warps:
 //   warps 0-3  softmax + epilogue of query tile 0 (one thread per row)
 //   warps 4-7  softmax + epilogue of query tile 1
 //   warp 8     TMA producer: Q tiles, then K_j, V_j into a ring of smem slots
@@ -34,12 +37,12 @@ namespace pa {
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kFwdThreads = 384;
 // Register split of the 384-thread block launched at 168 registers per thread
-// (384 x 168 = 64512): the two softmax warpgroups rise to 192, the producer /
-// MMA warpgroup drops to 120.  2*128*192 + 128*120 = 64512.  The build checks
+// (384 x 168 = 64512): the two softmax warpgroups rise to 224, the producer /
+// MMA warpgroup drops to 56.  2*128*224 + 128*56 = 64512.  The build checks
 // that the kernels are compiled at exactly kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 192;
-constexpr int kControlRegs = 120;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kFwdThreads * kLaunchRegs, "register split");
 
 template <int D>
@@ -64,6 +67,7 @@ struct FwdParams {
   const int32_t* cu;
   float* lse;
   const int32_t* counts;      // [0] items, [1] ordered segments
+  int32_t* next_item;         // work counter, zeroed by the scheduler kernel
   const int32_t* order;
   const int32_t* item_start;
   const uint8_t* maps;        // [B][4] tensor maps: q, k, v, out
@@ -79,7 +83,9 @@ struct Bars {
   uint64_t kv_full[8], kv_empty[8];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t epi_free[2], epi_full[2];
+  uint64_t sched_full[2], sched_empty[2];  // work-item hand-off from the producer
   uint64_t drain;
+  int32_t sched_item[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -129,13 +135,24 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
   using C = FwdCfg<D>;
   int slot = 0;
   uint32_t phase = 0;
-  uint32_t q_round = 0;
+  uint32_t q_round = 0, sk = 0;
   // last armed phase of every slot, for the drain after an abort
   uint32_t armed = 0, armed_phase = 0;
   bool q_armed = false;
   uint32_t q_armed_phase = 0;
   bool ok = true;
-  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+  for (;;) {
+    // hand the next item (or -1 = done) to the other warps
+    const int ss = sk & 1;
+    const uint32_t sph = (sk >> 1) & 1u;
+    ++sk;
+    if (!(ok = mbar_wait(&bars->sched_empty[ss], sph ^ 1u, wc))) break;
+    int32_t item = atomicAdd(p.next_item, 1);
+    if (item >= n_items) item = -1;
+    *reinterpret_cast<volatile int32_t*>(&bars->sched_item[ss]) = item;
+    mbar_arrive(&bars->sched_full[ss]);
+    if (item < 0) break;
+
     const WorkItem w = decode_item(item, p, n_sorted);
     const void* mq = seg_map(p, w.seg, 0);
     const void* mk = seg_map(p, w.seg, 1);
@@ -174,6 +191,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
         }
       }
     }
+    if (!ok) break;
   }
   if (!ok) {
     // Let every copy this thread started land before the CTA can exit.
@@ -184,39 +202,60 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
   }
 }
 
+// Takes the next item from the producer's hand-off ring; -1 when the work is done,
+// -2 when the wait gave up.  `arrive` releases the slot (one arrival per caller).
+__device__ __forceinline__ int32_t next_item_from_ring(Bars* bars, uint32_t& sk, const WaitCtl& wc, bool arrive) {
+  const int ss = sk & 1;
+  const uint32_t sph = (sk >> 1) & 1u;
+  ++sk;
+  if (!mbar_wait(&bars->sched_full[ss], sph, wc)) return -2;
+  const int32_t item = *reinterpret_cast<volatile int32_t*>(&bars->sched_item[ss]);
+  if (arrive) mbar_arrive(&bars->sched_empty[ss]);
+  return item;
+}
+
 // ------------------------------------------------------------------ MMA issuer
+// Unrolled issue loops over split descriptors: per MMA only the 32-bit start
+// addresses change (no carry leaves the 14-bit field: shared-memory addresses
+// are below 256 KB), the high word is one constant.
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+  constexpr uint32_t hi = sdesc_sw128_hi(1024);
+  const uint32_t a0 = sdesc_sw128_lo(q_addr, 16), b0 = sdesc_sw128_lo(k_addr, 16);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * FwdCfg<D>::kBlockBytes + (kk & 3) * 32;
-    mma_bf16_ss(d_tmem, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc,
-                kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * FwdCfg<D>::kBlockBytes + (kk & 3) * 32) >> 4;
+    mma_bf16_ss_lo(d_tmem, a0 + off, b0 + off, hi, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+  constexpr uint32_t hi = sdesc_sw128_hi(1024);
+  const uint32_t b0 = sdesc_sw128_lo(v_addr, FwdCfg<D>::kBlockBytes);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk) {
-    mma_bf16_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_addr + kk * 16 * 128, FwdCfg<D>::kBlockBytes, 1024), idesc,
-                (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < 128 / 16; ++kk)
+    mma_bf16_ts_lo(d_tmem, p_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
+                   (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
 __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, const WaitCtl& wc,
-                                        uint32_t tmem, int32_t n_items, int32_t n_sorted) {
+                                        uint32_t tmem, int32_t n_sorted) {
   using C = FwdCfg<D>;
   const uint32_t q_addr0 = smem_u32(smem + C::kOffQ);
   const uint32_t kv_addr0 = smem_u32(smem + C::kOffKV);
   int slot = 0;
   uint32_t phase = 0, q_round = 0;
   uint32_t p_ph = 0, oe_ph = 0;  // bit t: phase of tile t
+  uint32_t sk = 0;
   bool ok = true;
-  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+  for (;;) {
+    const int32_t item = next_item_from_ring(bars, sk, wc, true);
+    if (item == -2) ok = false;
+    if (item < 0) break;
     const WorkItem w = decode_item(item, p, n_sorted);
     if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
     ++q_round;
@@ -267,6 +306,7 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
         if (j + 2 == w.nkv) mma_commit(&bars->q_empty);
       }
     }
+    if (!ok) break;
   }
   // Every MMA issued so far completes before tensor memory is released.
   mma_commit(&bars->drain);
@@ -274,9 +314,79 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
 }
 
 // ------------------------------------------------------------------ softmax + epilogue
+// Row extreme of the 128 scores: max (kNeg = false) or min (kNeg = true, for a
+// negative scale), keys >= kv_valid excluded when kPartial.  Eight independent
+// chains of three-input max/min keep the dependency depth near 10.
+template <bool kPartial, bool kNeg>
+__device__ __forceinline__ float row_extreme(const uint32_t (&r)[128], int kv_valid) {
+  const float fill = kNeg ? INFINITY : -INFINITY;
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = fill;
+#pragma unroll
+  for (int k = 0; k < 128; k += 16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x0 = __uint_as_float(r[k + 2 * i]), x1 = __uint_as_float(r[k + 2 * i + 1]);
+      if (kPartial) {
+        x0 = (k + 2 * i < kv_valid) ? x0 : fill;
+        x1 = (k + 2 * i + 1 < kv_valid) ? x1 : fill;
+      }
+      a[i] = kNeg ? min3f(a[i], x0, x1) : max3f(a[i], x0, x1);
+    }
+  }
+  if (kNeg) return min3f(min3f(a[0], a[1], a[2]), min3f(a[3], a[4], a[5]), fminf(a[6], a[7]));
+  return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// One 128 x 128 score tile of one row (thread): row extreme, exponent-shift
+// update, P = exp2(s*c - m) -> bf16 into tensor memory, row sums.  Returns the
+// O rescale factor (1 when the shift did not move).
+template <bool kPartial, bool kNeg>
+__device__ __forceinline__ float softmax_tile(const uint32_t (&r)[128], int kv_valid, bool first, float c,
+                                              uint32_t tS, float& m, float& l, float& lr, bool& rescale) {
+  const float xmax = row_extreme<kPartial, kNeg>(r, kv_valid) * c;  // log2 units
+  float alpha = 1.0f;
+  rescale = false;
+  if (first) {
+    m = xmax;
+  } else if (__any_sync(0xffffffffu, xmax > m + kRescaleLog2)) {
+    const float m_new = fmaxf(m, xmax);
+    alpha = ex2_approx(m - m_new);
+    l *= alpha;
+    lr *= alpha;
+    m = m_new;
+    rescale = true;
+  }
+  const float neg_m = -m;
+  float su[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int k0 = cc * 32 + 2 * k;
+      float p0 = ex2_approx(fmaf(__uint_as_float(r[k0]), c, neg_m));
+      float p1 = ex2_approx(fmaf(__uint_as_float(r[k0 + 1]), c, neg_m));
+      if (kPartial) {
+        p0 = k0 < kv_valid ? p0 : 0.f;
+        p1 = k0 + 1 < kv_valid ? p1 : 0.f;
+      }
+      const uint32_t pr = pack_bf16x2(p0, p1);
+      su[k & 3] += p0 + p1;
+      sr[k & 3] += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
+      pk[k] = pr;
+    }
+    PA_TMEM_ST16(tS + cc * 16, pk);
+  }
+  l += (su[0] + su[1]) + (su[2] + su[3]);
+  lr += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+  return alpha;
+}
+
 template <int D>
 __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, Bars* bars, const WaitCtl& wc,
-                                            uint32_t tmem, int32_t n_items, int32_t n_sorted, int tile) {
+                                            uint32_t tmem, int32_t n_sorted, int tile) {
   using C = FwdCfg<D>;
   const int t = threadIdx.x & 127;  // row of the query tile
   const int lane = threadIdx.x & 31;
@@ -285,10 +395,16 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
   const uint32_t tO = tmem + lane_base + C::col_o(tile);
   uint8_t* stage = smem + C::kOffO + tile * C::kTileBytes;
   const float c = p.scale_log2;
-  uint32_t s_ph = 0, of_ph = 0, ef_ph = 0, eful_ph = 0;
+  uint32_t s_ph = 0, of_ph = 0, ef_ph = 0, eful_ph = 0, sk = 0;
   bool ok = true;
 
-  for (int32_t item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+  for (;;) {
+    int32_t item = next_item_from_ring(bars, sk, wc, false);
+    if (__any_sync(0xffffffffu, item == -2)) item = -2;
+    __syncwarp();
+    if (lane == 0 && item != -2) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
+    if (item == -2) ok = false;
+    if (item < 0) break;
     const WorkItem w = decode_item(item, p, n_sorted);
     if (tile == 1 && !w.two) continue;
     // l: sum of the fp32 exponentials (gives lse); lr: sum of the same values rounded to
@@ -306,61 +422,15 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
       PA_TMEM_LD32(tS + 64, (r + 64));
       PA_TMEM_LD32(tS + 96, (r + 96));
       tmem_wait_ld();
-      const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment (masked above)
-      const bool partial = kv_valid < 128;
-      float mx;
-      if (c >= 0.f) {
-        mx = -INFINITY;
-        if (!partial) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) mx = fmaxf(mx, k < kv_valid ? __uint_as_float(r[k]) : -INFINITY);
-        }
+      const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment
+      bool rescale;
+      float alpha;
+      if (kv_valid >= 128) {
+        alpha = c >= 0.f ? softmax_tile<false, false>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale)
+                         : softmax_tile<false, true>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale);
       } else {
-        mx = INFINITY;
-        if (!partial) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) mx = fminf(mx, __uint_as_float(r[k]));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 128; ++k) mx = fminf(mx, k < kv_valid ? __uint_as_float(r[k]) : INFINITY);
-        }
-      }
-      const float xmax = mx * c;  // largest scaled score of the row in this tile (log2 units)
-      float alpha = 1.0f;
-      bool rescale = false;
-      if (j == 0) {
-        m = xmax;
-      } else if (__any_sync(0xffffffffu, xmax > m + kRescaleLog2)) {
-        const float m_new = fmaxf(m, xmax);
-        alpha = ex2_approx(m - m_new);
-        l *= alpha;
-        lr *= alpha;
-        m = m_new;
-        rescale = true;
-      }
-      const float neg_m = -m;
-      float rs = 0.f, rsr = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int k0 = cc * 32 + 2 * k;
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[k0]), c, neg_m));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[k0 + 1]), c, neg_m));
-          if (partial) {
-            p0 = k0 < kv_valid ? p0 : 0.f;
-            p1 = k0 + 1 < kv_valid ? p1 : 0.f;
-          }
-          const uint32_t pr = pack_bf16x2(p0, p1);
-          rs += p0 + p1;
-          rsr += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
-          pk[k] = pr;
-        }
-        PA_TMEM_ST16(tS + cc * 16, pk);
+        alpha = c >= 0.f ? softmax_tile<true, false>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale)
+                         : softmax_tile<true, true>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale);
       }
       if (rescale) {
         // O += P V of the previous tile has completed (S of this tile was issued after it).
@@ -374,8 +444,6 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
           PA_TMEM_ST32(tO + cc * 32, o);
         }
       }
-      l += rs;
-      lr += rsr;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -463,6 +531,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_init(&bars->o_empty[t], 4);
       mbar_init(&bars->epi_free[t], 1);
       mbar_init(&bars->epi_full[t], 128);
+      mbar_init(&bars->sched_full[t], 1);
+      mbar_init(&bars->sched_empty[t], 9);  // the MMA thread + one lane of each softmax warp
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -482,7 +552,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   // barrier over the whole block, and only the tensor-memory owner continues.
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    run_softmax<D>(p, smem, bars, wc, tmem, n_items, n_sorted, warp >> 2);
+    run_softmax<D>(p, smem, bars, wc, tmem, n_sorted, warp >> 2);
     tc_fence_before();
     named_bar_sync(1, kFwdThreads);
   } else {
@@ -490,7 +560,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     if (warp == 8) {
       if ((threadIdx.x & 31) == 0) run_producer<D>(p, smem, bars, wc, n_items, n_sorted);
     } else if (warp == 9) {
-      if ((threadIdx.x & 31) == 0) run_mma<D>(p, smem, bars, wc, tmem, n_items, n_sorted);
+      if ((threadIdx.x & 31) == 0) run_mma<D>(p, smem, bars, wc, tmem, n_sorted);
     }
     __syncwarp();
     tc_fence_before();

@@ -214,6 +214,7 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
   fp.cu = cu_seqlens;
   fp.lse = lse;
   fp.counts = sp.counts;
+  fp.next_item = sp.counts + 2;
   fp.order = sp.order;
   fp.item_start = sp.item_start;
   fp.maps = sp.maps;

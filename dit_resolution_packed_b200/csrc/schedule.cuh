@@ -36,7 +36,7 @@ struct SchedParams {
   const void* base[4];     // q, k, v, out base pointers
   const int32_t* cu;       // [B+1]
   int32_t* status;         // status word
-  int32_t* counts;         // [0] = work items, [1] = non-empty segments
+  int32_t* counts;         // [0] = work items, [1] = non-empty segments, [2] = work counter (zeroed)
   int32_t* order;          // [B] segment ids, longest first
   int32_t* item_start;     // [B+1] first item of each ordered segment
   uint8_t* maps;           // [B][4] tensor maps, 128 bytes each
@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       atomicCAS(p.status, 0, s_bad == 2 ? p.err_cu : p.err_max);
       p.counts[0] = 0;
       p.counts[1] = 0;
+      p.counts[2] = 0;
     }
     return;
   }
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     p.item_start[n_sorted] = static_cast<int32_t>(carry);
     p.counts[0] = static_cast<int32_t>(carry);
     p.counts[1] = n_sorted;
+    p.counts[2] = 0;
   }
 
   // 4. per-segment tensor maps: copy the template, then move its base and row extent
