@@ -1,6 +1,6 @@
 // attn_fwd_sm100.cuh -- packed variable-length bidirectional attention forward
 // for B200 (sm_100a): TMA tile loads, tcgen05 MMAs accumulating in tensor
-// memory, online softmax in registers, TMA stores of the output.
+// memory, online softmax in registers, 16-byte row stores of the output.
 //
 // Math (SparseAttn page, section 3.1; GigaPath-Flash page, sections 3.2/4.2 for
 // the blockwise online softmax): per query row, with x = scale*log2(e)*q.k,
@@ -52,11 +52,10 @@ struct FwdCfg {
   static constexpr int kTileBytes = kRows * D * 2;       // bf16 tile
   static constexpr int kColBlocks = D / 64;              // 128-byte swizzle atoms across d
   static constexpr int kBlockBytes = kRows * 128;        // one 64-column block of a tile
-  static constexpr int kSlots = (D == 128) ? 3 : 6;      // K/V ring depth
+  static constexpr int kSlots = (D == 128) ? 5 : 10;     // K/V ring depth (tiles)
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffO = kOffKV + kSlots * kTileBytes;
-  static constexpr int kOffBar = kOffO + 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // + 1024 for base alignment
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t col_s(int tile) { return tile ? 128u : 0u; }
@@ -65,12 +64,13 @@ struct FwdCfg {
 
 struct FwdParams {
   const int32_t* cu;
+  void* out;                  // bf16 [T, H, d]
   float* lse;
   const int32_t* counts;      // [0] items, [1] ordered segments
   int32_t* next_item;         // work counter, zeroed by the scheduler kernel
   const int32_t* order;
   const int32_t* item_start;
-  const uint8_t* maps;        // [B][4] tensor maps: q, k, v, out
+  const uint8_t* maps;        // [B][3] tensor maps: q, k, v
   int32_t* status;
   int32_t heads;
   float scale_log2;           // scale * log2(e)
@@ -80,9 +80,9 @@ struct FwdParams {
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[8], kv_empty[8];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t epi_free[2], epi_full[2];
+  uint64_t kv_full[12], kv_empty[12];
+  uint64_t s_full[2], o_full[2], o_empty[2];
+  uint64_t p_full[2][2];  // [tile][half]: P columns of keys 0-63 / 64-127 are in tensor memory
   uint64_t sched_full[2], sched_empty[2];  // work-item hand-off from the producer
   uint64_t drain;
   int32_t sched_item[2];
@@ -115,7 +115,7 @@ __device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p
 }
 
 __device__ __forceinline__ const void* seg_map(const FwdParams& p, int32_t seg, int which) {
-  return p.maps + (static_cast<size_t>(seg) * 4 + which) * 128;
+  return p.maps + (static_cast<size_t>(seg) * 3 + which) * 128;
 }
 
 // A wait used while draining after an abort: ignores the abort flag, bounded by its own limit.
@@ -230,15 +230,19 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32
   }
 }
 
+// O (+)= P V over the keys [64*half, 64*half + 64) of the tile.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, int half,
+                                              bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
   const uint32_t b0 = sdesc_sw128_lo(v_addr, FwdCfg<D>::kBlockBytes);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk)
+  for (int kq = 0; kq < 4; ++kq) {
+    const int kk = half * 4 + kq;
     mma_bf16_ts_lo(d_tmem, p_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
                    (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <int D>
@@ -276,11 +280,6 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
       const int vs = slot;
       if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
       if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
-      if (has_next) {
-        ks = slot;
-        if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
-        if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
-      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (t == 1 && !w.two) break;
@@ -288,11 +287,20 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
           if (!(ok = mbar_wait(&bars->o_empty[t], ((oe_ph >> t) & 1u) ^ 1u, wc))) break;
           oe_ph ^= 1u << t;
         }
-        if (!(ok = mbar_wait(&bars->p_full[t], (p_ph >> t) & 1u, wc))) break;
+        if (!(ok = mbar_wait(&bars->p_full[t][0], (p_ph >> t) & 1u, wc))) break;
+        tc_fence_after();
+        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, 0, j > 0);
+        if (!(ok = mbar_wait(&bars->p_full[t][1], (p_ph >> t) & 1u, wc))) break;
         p_ph ^= 1u << t;
         tc_fence_after();
-        issue_pv<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, j > 0);
+        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, 1, true);
         if (has_next) {
+          if (t == 0) {  // K_{j+1} is needed only now, after P.V of tile 0 is queued
+            ks = slot;
+            if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
+            if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
+            tc_fence_after();
+          }
           issue_s<D>(tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
           mma_commit(&bars->s_full[t]);
         } else {
@@ -314,23 +322,24 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
 }
 
 // ------------------------------------------------------------------ softmax + epilogue
-// Row extreme of the 128 scores: max (kNeg = false) or min (kNeg = true, for a
-// negative scale), keys >= kv_valid excluded when kPartial.  Eight independent
-// chains of three-input max/min keep the dependency depth near 10.
+// Row extreme of the 128 scores (64 register pairs): max (kNeg = false) or min
+// (kNeg = true, for a negative scale), keys >= kv_valid excluded when kPartial.
+// Eight independent chains of three-input max/min keep the dependency depth
+// near 10.
 template <bool kPartial, bool kNeg>
-__device__ __forceinline__ float row_extreme(const uint32_t (&r)[128], int kv_valid) {
+__device__ __forceinline__ float row_extreme(const uint64_t (&v)[64], int kv_valid) {
   const float fill = kNeg ? INFINITY : -INFINITY;
   float a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = fill;
 #pragma unroll
-  for (int k = 0; k < 128; k += 16) {
+  for (int k = 0; k < 64; k += 8) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float x0 = __uint_as_float(r[k + 2 * i]), x1 = __uint_as_float(r[k + 2 * i + 1]);
+      float x0 = f2_lo(v[k + i]), x1 = f2_hi(v[k + i]);
       if (kPartial) {
-        x0 = (k + 2 * i < kv_valid) ? x0 : fill;
-        x1 = (k + 2 * i + 1 < kv_valid) ? x1 : fill;
+        x0 = (2 * (k + i) < kv_valid) ? x0 : fill;
+        x1 = (2 * (k + i) + 1 < kv_valid) ? x1 : fill;
       }
       a[i] = kNeg ? min3f(a[i], x0, x1) : max3f(a[i], x0, x1);
     }
@@ -340,48 +349,65 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&r)[128], int kv_va
 }
 
 // One 128 x 128 score tile of one row (thread): row extreme, exponent-shift
-// update, P = exp2(s*c - m) -> bf16 into tensor memory, row sums.  Returns the
-// O rescale factor (1 when the shift did not move).
-template <bool kPartial, bool kNeg>
-__device__ __forceinline__ float softmax_tile(const uint32_t (&r)[128], int kv_valid, bool first, float c,
-                                              uint32_t tS, float& m, float& l, float& lr, bool& rescale) {
-  const float xmax = row_extreme<kPartial, kNeg>(r, kv_valid) * c;  // log2 units
-  float alpha = 1.0f;
-  rescale = false;
+// update (rescaling O first when it moves), then P = exp2(s*c - m) -> bf16 into
+// tensor memory in two halves of 64 keys; each half is handed to the MMA warp
+// as soon as it is stored, so P.V of keys 0-63 overlaps the exponentials of
+// keys 64-127.  Scores stay in register pairs and use packed fp32 arithmetic.
+template <bool kPartial, bool kNeg, int D>
+__device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_valid, bool first, float c,
+                                             uint32_t tS, uint32_t tO, float& m, float& l, float& lr,
+                                             uint64_t* p_full_half, int lane) {
+  const float xmax = row_extreme<kPartial, kNeg>(v, kv_valid) * c;  // log2 units
   if (first) {
     m = xmax;
   } else if (__any_sync(0xffffffffu, xmax > m + kRescaleLog2)) {
     const float m_new = fmaxf(m, xmax);
-    alpha = ex2_approx(m - m_new);
+    const float alpha = ex2_approx(m - m_new);
     l *= alpha;
     lr *= alpha;
     m = m_new;
-    rescale = true;
-  }
-  const float neg_m = -m;
-  float su[4] = {0.f, 0.f, 0.f, 0.f}, sr[4] = {0.f, 0.f, 0.f, 0.f};
+    // O += P V of the previous tile has completed (S of this tile was issued after it).
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    uint32_t pk[16];
+    for (int cc = 0; cc < D / 16; ++cc) {
+      uint32_t o[16];
+      PA_TMEM_LD16(tO + cc * 16, o);
+      tmem_wait_ld();
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int k0 = cc * 32 + 2 * k;
-      float p0 = ex2_approx(fmaf(__uint_as_float(r[k0]), c, neg_m));
-      float p1 = ex2_approx(fmaf(__uint_as_float(r[k0 + 1]), c, neg_m));
-      if (kPartial) {
-        p0 = k0 < kv_valid ? p0 : 0.f;
-        p1 = k0 + 1 < kv_valid ? p1 : 0.f;
-      }
-      const uint32_t pr = pack_bf16x2(p0, p1);
-      su[k & 3] += p0 + p1;
-      sr[k & 3] += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
-      pk[k] = pr;
+      for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+      PA_TMEM_ST16(tO + cc * 16, o);
     }
-    PA_TMEM_ST16(tS + cc * 16, pk);
   }
-  l += (su[0] + su[1]) + (su[2] + su[3]);
-  lr += (sr[0] + sr[1]) + (sr[2] + sr[3]);
-  return alpha;
+  const uint64_t c2 = f2_pack(c, c);
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t su[2] = {0, 0}, sr[2] = {0, 0};  // packed partial sums (0.0f bit patterns)
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int i = cc * 16 + k;  // pair index: keys 2i, 2i+1
+        uint64_t x = f2_fma(v[i], c2, negm2);
+        if (kPartial) {
+          x = f2_pack(2 * i < kv_valid ? f2_lo(x) : -INFINITY, 2 * i + 1 < kv_valid ? f2_hi(x) : -INFINITY);
+        }
+        const uint64_t pp = ex2x2(x);
+        const uint32_t pr = pack_bf16x2_pair(pp);
+        su[k & 1] = f2_add(su[k & 1], pp);
+        sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
+        pk[k] = pr;
+      }
+      PA_TMEM_ST16(tS + cc * 16, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&p_full_half[half]);
+  }
+  const uint64_t su2 = f2_add(su[0], su[1]), sr2 = f2_add(sr[0], sr[1]);
+  l += f2_lo(su2) + f2_hi(su2);
+  lr += f2_lo(sr2) + f2_hi(sr2);
 }
 
 template <int D>
@@ -393,9 +419,8 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
   const uint32_t tS = tmem + lane_base + C::col_s(tile);
   const uint32_t tO = tmem + lane_base + C::col_o(tile);
-  uint8_t* stage = smem + C::kOffO + tile * C::kTileBytes;
   const float c = p.scale_log2;
-  uint32_t s_ph = 0, of_ph = 0, ef_ph = 0, eful_ph = 0, sk = 0;
+  uint32_t s_ph = 0, of_ph = 0, sk = 0;
   bool ok = true;
 
   for (;;) {
@@ -416,60 +441,36 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       s_ph ^= 1u;
       tc_fence_after();
-      uint32_t r[128];
-      PA_TMEM_LD32(tS + 0, (r + 0));
-      PA_TMEM_LD32(tS + 32, (r + 32));
-      PA_TMEM_LD32(tS + 64, (r + 64));
-      PA_TMEM_LD32(tS + 96, (r + 96));
-      tmem_wait_ld();
+      uint64_t r[64];
+      tmem_ld128_pairs(tS, r);
       const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment
-      bool rescale;
-      float alpha;
+      uint64_t* ph = bars->p_full[tile];
       if (kv_valid >= 128) {
-        alpha = c >= 0.f ? softmax_tile<false, false>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale)
-                         : softmax_tile<false, true>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale);
+        if (c >= 0.f) softmax_tile<false, false, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        else softmax_tile<false, true, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
       } else {
-        alpha = c >= 0.f ? softmax_tile<true, false>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale)
-                         : softmax_tile<true, true>(r, kv_valid, j == 0, c, tS, m, l, lr, rescale);
+        if (c >= 0.f) softmax_tile<true, false, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        else softmax_tile<true, true, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
       }
-      if (rescale) {
-        // O += P V of the previous tile has completed (S of this tile was issued after it).
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          PA_TMEM_LD32(tO + cc * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          PA_TMEM_ST32(tO + cc * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[tile]);
     }
     if (!ok) break;
 
-    // ---- epilogue: O / l -> bf16 -> swizzled staging tile -> TMA store (clipped at the segment end)
+    // ---- epilogue: O / l -> bf16 -> 16-byte stores of this thread's row (rows past the
+    // segment end are not written); lse from the unrounded sum.
     ok = mbar_wait(&bars->o_full[tile], of_ph, wc);
     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
     of_ph ^= 1u;
     tc_fence_after();
-    if (t == 0) {
-      bulk_wait_group_read0();  // the previous store has finished reading the staging tile
-      mbar_arrive(&bars->epi_free[tile]);
-    }
-    ok = mbar_wait(&bars->epi_free[tile], ef_ph, wc);
-    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-    ef_ph ^= 1u;
+    const int32_t row = w.q0 + tile * 128 + t;
+    const bool row_ok = row < w.len;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                                          (static_cast<size_t>(w.beg + (row_ok ? row : 0)) * p.heads + w.head) * D);
     const float inv_l = 1.0f / lr;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
       PA_TMEM_LD32(tO + cc * 32, o);
       tmem_wait_ld();
-      uint8_t* row = stage + (cc >> 1) * C::kBlockBytes + t * 128;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint4 v;
@@ -477,34 +478,17 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
         v.y = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2]) * inv_l, __uint_as_float(o[q4 * 8 + 3]) * inv_l);
         v.z = pack_bf16x2(__uint_as_float(o[q4 * 8 + 4]) * inv_l, __uint_as_float(o[q4 * 8 + 5]) * inv_l);
         v.w = pack_bf16x2(__uint_as_float(o[q4 * 8 + 6]) * inv_l, __uint_as_float(o[q4 * 8 + 7]) * inv_l);
-        const int chunk = (cc & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-        *reinterpret_cast<uint4*>(row + ((chunk ^ (t & 7)) << 4)) = v;
+        if (row_ok) dst[cc * 4 + q4] = v;
       }
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->o_empty[tile]);  // O columns may be overwritten now
-    fence_proxy_async_smem();
-    mbar_arrive(&bars->epi_full[tile]);
-    const int32_t row0 = w.q0 + tile * 128;
-    if (t == 0) {
-      // A failed wait here only skips the store; the abort flag stops every role at its next wait.
-      if (mbar_wait(&bars->epi_full[tile], eful_ph, wc)) {
-        const void* mo = seg_map(p, w.seg, 3);
-        fence_tmap_acquire(mo);
-#pragma unroll
-        for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_store_2d(mo, w.head * D + cb * 64, row0, stage + cb * C::kBlockBytes);
-        bulk_commit_group();
-      }
-    }
-    eful_ph ^= 1u;
-    if (row0 + t < w.len) {
+    if (row_ok) {
       const float lse2 = m + __log2f(l);
-      p.lse[static_cast<size_t>(w.beg + row0 + t) * p.heads + w.head] = lse2 * 0.69314718055994531f;
+      p.lse[static_cast<size_t>(w.beg + row) * p.heads + w.head] = lse2 * 0.69314718055994531f;
     }
   }
-  if (t == 0) bulk_wait_group0();
 }
 
 template <int D>
@@ -526,11 +510,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 4);
+      mbar_init(&bars->p_full[t][0], 4);
+      mbar_init(&bars->p_full[t][1], 4);
       mbar_init(&bars->o_full[t], 1);
       mbar_init(&bars->o_empty[t], 4);
-      mbar_init(&bars->epi_free[t], 1);
-      mbar_init(&bars->epi_full[t], 128);
       mbar_init(&bars->sched_full[t], 1);
       mbar_init(&bars->sched_empty[t], 9);  // the MMA thread + one lane of each softmax warp
     }

@@ -1,8 +1,8 @@
 // packattn.cu -- host side of the C ABI declared in include/packattn.h.
 //
 // A call validates its arguments on the host, finds (or grows) the workspace of
-// its (device, stream) pair, encodes four template tensor maps over the whole
-// q / k / v / out matrices, and enqueues two kernels on the caller's stream:
+// its (device, stream) pair, encodes three template tensor maps over the whole
+// q / k / v matrices, and enqueues two kernels on the caller's stream:
 // the segment scheduler (one CTA) and the persistent attention kernel (one CTA
 // per SM).  Nothing synchronises on this path.
 #include <cuda.h>
@@ -73,7 +73,7 @@ WsLayout ws_layout(int32_t batch) {
   L.order = 128;
   L.item_start = align_up(L.order + 4 * static_cast<size_t>(batch), 128);
   L.maps = align_up(L.item_start + 4 * (static_cast<size_t>(batch) + 1), 128);
-  L.total = L.maps + 512 * static_cast<size_t>(batch);
+  L.total = L.maps + 384 * static_cast<size_t>(batch);
   return L;
 }
 
@@ -189,8 +189,8 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
 
   pa::SchedParams sp;
   std::memset(&sp, 0, sizeof(sp));
-  const void* bases[4] = {q, k, v, out};
-  for (int i = 0; i < 4; ++i) {
+  const void* bases[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
     if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
     sp.base[i] = bases[i];
   }
@@ -212,6 +212,7 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
 
   pa::FwdParams fp;
   fp.cu = cu_seqlens;
+  fp.out = out;
   fp.lse = lse;
   fp.counts = sp.counts;
   fp.next_item = sp.counts + 2;

@@ -11,10 +11,10 @@
 //   3. publishes, in that order, the first work-item index of every segment;
 //      a segment of L tokens holds heads * ceil(L / 256) items, one per
 //      (head, pair of 128-row query tiles);
-//   4. writes four tensor maps per segment (q, k, v, out) whose base is the
+//   4. writes three tensor maps per segment (q, k, v) whose base is the
 //      segment's first token and whose row extent is L, so that every TMA tile
-//      stops at the segment boundary: loads past it read zeros, stores past it
-//      are dropped, and no tile touches another image.
+//      stops at the segment boundary: loads past it read zeros and no tile
+//      touches another image.
 //
 // The mask of the method (Mage-Flow page, "Packing + Flash Attention varlen":
 // images attend only to themselves, no padding) is thereby carried entirely by
@@ -32,14 +32,14 @@ constexpr int kSchedThreads = 1024;
 constexpr int kSortBuckets = 4096;  // tile counts >= 4095 share the first bucket
 
 struct SchedParams {
-  CUtensorMap tmpl[4];     // q, k, v, out over the whole [T, H*d] matrix (host-encoded)
-  const void* base[4];     // q, k, v, out base pointers
+  CUtensorMap tmpl[3];     // q, k, v over the whole [T, H*d] matrix (host-encoded)
+  const void* base[3];     // q, k, v base pointers
   const int32_t* cu;       // [B+1]
   int32_t* status;         // status word
   int32_t* counts;         // [0] = work items, [1] = non-empty segments, [2] = work counter (zeroed)
   int32_t* order;          // [B] segment ids, longest first
   int32_t* item_start;     // [B+1] first item of each ordered segment
-  uint8_t* maps;           // [B][4] tensor maps, 128 bytes each
+  uint8_t* maps;           // [B][3] tensor maps, 128 bytes each
   uint64_t row_bytes;      // H * d * 2
   int32_t batch, total, heads, max_seqlen;
   int32_t err_cu, err_max;  // status codes to record
@@ -177,8 +177,8 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   }
 
   // 4. per-segment tensor maps: copy the template, then move its base and row extent
-  for (int idx = tid; idx < 4 * B; idx += kSchedThreads) {
-    const int s = idx >> 2, which = idx & 3;
+  for (int idx = tid; idx < 3 * B; idx += kSchedThreads) {
+    const int s = idx / 3, which = idx - 3 * s;
     const int32_t beg = p.cu[s], len = p.cu[s + 1] - beg;
     if (len <= 0) continue;
     uint8_t* dst = p.maps + static_cast<size_t>(idx) * 128;

@@ -254,6 +254,13 @@ __host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo_bytes) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])   \
       : "r"(taddr))
 
+#define PA_TMEM_LD16(taddr, r)                                                                                 \
+  asm volatile(                                                                                                \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"   \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),        \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])   \
+      : "r"(taddr))
+
 #define PA_TMEM_ST16(taddr, r)                                                                                 \
   asm volatile(                                                                                                \
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" \
@@ -270,6 +277,86 @@ __host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo_bytes) {
       "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),            \
       "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                                     \
       : "memory")
+
+// Loads 128 consecutive 32-bit columns of this thread's tensor-memory lane into
+// 64 register pairs (column 2i in the low half of pair i), waiting once for all.
+__device__ __forceinline__ void tmem_ld128_pairs(uint32_t taddr, uint64_t (&v)[64]) {
+  asm volatile(
+      "{\n\t.reg .b32 t<128>;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {t32, t33, t34, t35, t36, t37, t38, t39, t40, t41, t42, t43, t44, t45, t46, t47, t48, t49, t50, t51, t52, t53, t54, t55, t56, t57, t58, t59, t60, t61, t62, t63}, [%65];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {t64, t65, t66, t67, t68, t69, t70, t71, t72, t73, t74, t75, t76, t77, t78, t79, t80, t81, t82, t83, t84, t85, t86, t87, t88, t89, t90, t91, t92, t93, t94, t95}, [%66];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {t96, t97, t98, t99, t100, t101, t102, t103, t104, t105, t106, t107, t108, t109, t110, t111, t112, t113, t114, t115, t116, t117, t118, t119, t120, t121, t122, t123, t124, t125, t126, t127}, [%67];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "mov.b64 %0, {t0, t1};\n\t"
+      "mov.b64 %1, {t2, t3};\n\t"
+      "mov.b64 %2, {t4, t5};\n\t"
+      "mov.b64 %3, {t6, t7};\n\t"
+      "mov.b64 %4, {t8, t9};\n\t"
+      "mov.b64 %5, {t10, t11};\n\t"
+      "mov.b64 %6, {t12, t13};\n\t"
+      "mov.b64 %7, {t14, t15};\n\t"
+      "mov.b64 %8, {t16, t17};\n\t"
+      "mov.b64 %9, {t18, t19};\n\t"
+      "mov.b64 %10, {t20, t21};\n\t"
+      "mov.b64 %11, {t22, t23};\n\t"
+      "mov.b64 %12, {t24, t25};\n\t"
+      "mov.b64 %13, {t26, t27};\n\t"
+      "mov.b64 %14, {t28, t29};\n\t"
+      "mov.b64 %15, {t30, t31};\n\t"
+      "mov.b64 %16, {t32, t33};\n\t"
+      "mov.b64 %17, {t34, t35};\n\t"
+      "mov.b64 %18, {t36, t37};\n\t"
+      "mov.b64 %19, {t38, t39};\n\t"
+      "mov.b64 %20, {t40, t41};\n\t"
+      "mov.b64 %21, {t42, t43};\n\t"
+      "mov.b64 %22, {t44, t45};\n\t"
+      "mov.b64 %23, {t46, t47};\n\t"
+      "mov.b64 %24, {t48, t49};\n\t"
+      "mov.b64 %25, {t50, t51};\n\t"
+      "mov.b64 %26, {t52, t53};\n\t"
+      "mov.b64 %27, {t54, t55};\n\t"
+      "mov.b64 %28, {t56, t57};\n\t"
+      "mov.b64 %29, {t58, t59};\n\t"
+      "mov.b64 %30, {t60, t61};\n\t"
+      "mov.b64 %31, {t62, t63};\n\t"
+      "mov.b64 %32, {t64, t65};\n\t"
+      "mov.b64 %33, {t66, t67};\n\t"
+      "mov.b64 %34, {t68, t69};\n\t"
+      "mov.b64 %35, {t70, t71};\n\t"
+      "mov.b64 %36, {t72, t73};\n\t"
+      "mov.b64 %37, {t74, t75};\n\t"
+      "mov.b64 %38, {t76, t77};\n\t"
+      "mov.b64 %39, {t78, t79};\n\t"
+      "mov.b64 %40, {t80, t81};\n\t"
+      "mov.b64 %41, {t82, t83};\n\t"
+      "mov.b64 %42, {t84, t85};\n\t"
+      "mov.b64 %43, {t86, t87};\n\t"
+      "mov.b64 %44, {t88, t89};\n\t"
+      "mov.b64 %45, {t90, t91};\n\t"
+      "mov.b64 %46, {t92, t93};\n\t"
+      "mov.b64 %47, {t94, t95};\n\t"
+      "mov.b64 %48, {t96, t97};\n\t"
+      "mov.b64 %49, {t98, t99};\n\t"
+      "mov.b64 %50, {t100, t101};\n\t"
+      "mov.b64 %51, {t102, t103};\n\t"
+      "mov.b64 %52, {t104, t105};\n\t"
+      "mov.b64 %53, {t106, t107};\n\t"
+      "mov.b64 %54, {t108, t109};\n\t"
+      "mov.b64 %55, {t110, t111};\n\t"
+      "mov.b64 %56, {t112, t113};\n\t"
+      "mov.b64 %57, {t114, t115};\n\t"
+      "mov.b64 %58, {t116, t117};\n\t"
+      "mov.b64 %59, {t118, t119};\n\t"
+      "mov.b64 %60, {t120, t121};\n\t"
+      "mov.b64 %61, {t122, t123};\n\t"
+      "mov.b64 %62, {t124, t125};\n\t"
+      "mov.b64 %63, {t126, t127};\n\t"
+      "}\n"
+      : "=l"(v[0]), "=l"(v[1]), "=l"(v[2]), "=l"(v[3]), "=l"(v[4]), "=l"(v[5]), "=l"(v[6]), "=l"(v[7]), "=l"(v[8]), "=l"(v[9]), "=l"(v[10]), "=l"(v[11]), "=l"(v[12]), "=l"(v[13]), "=l"(v[14]), "=l"(v[15]), "=l"(v[16]), "=l"(v[17]), "=l"(v[18]), "=l"(v[19]), "=l"(v[20]), "=l"(v[21]), "=l"(v[22]), "=l"(v[23]), "=l"(v[24]), "=l"(v[25]), "=l"(v[26]), "=l"(v[27]), "=l"(v[28]), "=l"(v[29]), "=l"(v[30]), "=l"(v[31]), "=l"(v[32]), "=l"(v[33]), "=l"(v[34]), "=l"(v[35]), "=l"(v[36]), "=l"(v[37]), "=l"(v[38]), "=l"(v[39]), "=l"(v[40]), "=l"(v[41]), "=l"(v[42]), "=l"(v[43]), "=l"(v[44]), "=l"(v[45]), "=l"(v[46]), "=l"(v[47]), "=l"(v[48]), "=l"(v[49]), "=l"(v[50]), "=l"(v[51]), "=l"(v[52]), "=l"(v[53]), "=l"(v[54]), "=l"(v[55]), "=l"(v[56]), "=l"(v[57]), "=l"(v[58]), "=l"(v[59]), "=l"(v[60]), "=l"(v[61]), "=l"(v[62]), "=l"(v[63])
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+}
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -300,6 +387,41 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2 of both lanes of a pair (MUFU), result as a pair.
+__device__ __forceinline__ uint64_t ex2x2(uint64_t x) {
+  uint64_t y;
+  asm("{\n\t.reg .f32 a, b, c, d;\n\t"
+      "mov.b64 {a, b}, %1;\n\t"
+      "ex2.approx.ftz.f32 c, a;\n\t"
+      "ex2.approx.ftz.f32 d, b;\n\t"
+      "mov.b64 %0, {c, d};\n\t}"
+      : "=l"(y)
+      : "l"(x));
+  return y;
+}
+// bf16x2 of a pair (low lane -> low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2_pair(uint64_t x) {
+  uint32_t r;
+  asm("{\n\t.reg .f32 a, b;\n\t"
+      "mov.b64 {a, b}, %1;\n\t"
+      "cvt.rn.bf16x2.f32 %0, b, a;\n\t}"
+      : "=r"(r)
+      : "l"(x));
+  return r;
+}
+// acc += (fp32 value of the low bf16 of p, fp32 value of the high bf16 of p), lane-wise.
+__device__ __forceinline__ uint64_t add_bf16x2_as_f32x2(uint64_t acc, uint32_t p) {
+  uint64_t d;
+  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
+      "shl.b32 lo, %2, 16;\n\t"
+      "and.b32 hi, %2, 0xffff0000;\n\t"
+      "mov.b64 w, {lo, hi};\n\t"
+      "add.rn.f32x2 %0, %1, w;\n\t}"
+      : "=l"(d)
+      : "l"(acc), "r"(p));
   return d;
 }
 
