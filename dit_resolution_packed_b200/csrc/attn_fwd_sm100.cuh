@@ -35,6 +35,11 @@
 namespace pa {
 
 constexpr float kRescaleLog2 = 8.0f;
+// In every group of four key pairs of a full score tile, this many are
+// exponentiated on the FMA pipe (polynomial) instead of the MUFU unit.
+// Measured on B200: 1 of 4 costs 8-10 % at d = 128 (issue slots, not MUFU,
+// bound this softmax), so it is off.
+constexpr int kPolyPairsPer4 = 0;
 constexpr int kFwdThreads = 384;
 // Register split of the 384-thread block launched at 168 registers per thread
 // (384 x 168 = 64512): the two softmax warpgroups rise to 224, the producer /
@@ -379,6 +384,9 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
   }
   const uint64_t c2 = f2_pack(c, c);
   const uint64_t negm2 = f2_pack(-m, -m);
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  const Exp2PolyConsts ek{f2_pack(magic, magic), f2_pack(-magic, -magic), f2_pack(kExp2C0, kExp2C0),
+                          f2_pack(kExp2C1, kExp2C1), f2_pack(kExp2C2, kExp2C2), f2_pack(kExp2C3, kExp2C3)};
   uint64_t su[2] = {0, 0}, sr[2] = {0, 0};  // packed partial sums (0.0f bit patterns)
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -392,7 +400,7 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
         if (kPartial) {
           x = f2_pack(2 * i < kv_valid ? f2_lo(x) : -INFINITY, 2 * i + 1 < kv_valid ? f2_hi(x) : -INFINITY);
         }
-        const uint64_t pp = ex2x2(x);
+        const uint64_t pp = (!kPartial && (k & 3) >= 4 - kPolyPairsPer4) ? ex2x2_poly(x, ek) : ex2x2(x);
         const uint32_t pr = pack_bf16x2_pair(pp);
         su[k & 1] = f2_add(su[k & 1], pp);
         sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);

@@ -8,6 +8,8 @@
 #pragma once
 #include <cstdint>
 
+#include "exp2_poly.cuh"
+
 namespace pa {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -402,6 +404,39 @@ __device__ __forceinline__ uint64_t ex2x2(uint64_t x) {
       : "l"(x));
   return y;
 }
+// exp2 of both lanes of a pair on the FMA pipe (no MUFU): Cody-Waite style
+// reduction x = n + f, n = round(x) by the 1.5*2^23 addition trick, |f| <= 1/2,
+// then 2^f by the degree-3 minimax polynomial of exp2_poly.cuh (Horner, packed
+// fma) and 2^n by adding n to the exponent field.  Inputs are clamped to
+// >= -125 so that 2^n stays a normal number; the result is then < 2^-124,
+// negligible against the row sum (>= 1).  Max relative error ~7.5e-5.
+// `k` holds the pair constants: {magic, magic}, {-magic, -magic}, C0..C3 pairs.
+struct Exp2PolyConsts {
+  uint64_t magic, neg_magic, c0, c1, c2, c3;
+};
+__device__ __forceinline__ uint64_t ex2x2_poly(uint64_t x, const Exp2PolyConsts& k) {
+  uint64_t y;
+  asm("{\n\t.reg .f32 a, b;\n\t.reg .b64 xc, t, n, f, p;\n\t.reg .b32 tl, th, pl, ph, rl, rh;\n\t"
+      "mov.b64 {a, b}, %1;\n\t"
+      "max.f32 a, a, 0fC2FA0000;\n\t"  // -125
+      "max.f32 b, b, 0fC2FA0000;\n\t"
+      "mov.b64 xc, {a, b};\n\t"
+      "add.rn.f32x2 t, xc, %2;\n\t"      // t = x + magic: round(x) in the low mantissa bits
+      "add.rn.f32x2 n, t, %3;\n\t"       // n = round(x) as a float
+      "sub.rn.f32x2 f, xc, n;\n\t"       // f = x - n, |f| <= 1/2
+      "fma.rn.f32x2 p, %7, f, %6;\n\t"   // C3 f + C2
+      "fma.rn.f32x2 p, p, f, %5;\n\t"    // (..) f + C1
+      "fma.rn.f32x2 p, p, f, %4;\n\t"    // (..) f + C0
+      "mov.b64 {tl, th}, t;\n\t"
+      "mov.b64 {pl, ph}, p;\n\t"
+      "mad.lo.u32 rl, tl, 8388608, pl;\n\t"  // exponent += n (bits of t hold n mod 2^9)
+      "mad.lo.u32 rh, th, 8388608, ph;\n\t"
+      "mov.b64 %0, {rl, rh};\n\t}"
+      : "=l"(y)
+      : "l"(x), "l"(k.magic), "l"(k.neg_magic), "l"(k.c0), "l"(k.c1), "l"(k.c2), "l"(k.c3));
+  return y;
+}
+
 // bf16x2 of a pair (low lane -> low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2_pair(uint64_t x) {
   uint32_t r;
