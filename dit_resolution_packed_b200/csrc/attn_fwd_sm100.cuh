@@ -506,8 +506,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   const int warp = threadIdx.x >> 5;
-  const int32_t n_items = p.counts[0];
-  const int32_t n_sorted = p.counts[1];
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -538,6 +536,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const WaitCtl wc{&bars->abort_flag, p.status, p.wait_limit_ns, p.err_timeout};
+  // Everything above overlaps the schedule kernel (programmatic dependent
+  // launch); the work list, the tensor maps and the counters are read only
+  // after it has completed.
+  pdl_wait_primary();
+  const int32_t n_items = p.counts[0];
+  const int32_t n_sorted = p.counts[1];
 
   // The two register regions never merge again: each branch ends with its own
   // barrier over the whole block, and only the tensor-memory owner continues.

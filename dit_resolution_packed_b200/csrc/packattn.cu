@@ -238,11 +238,21 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
     ++g_prof_used;
     cudaEventRecord(ev0, stream);
   }
-  if (head_dim == 128)
-    pa::attn_fwd_kernel<128><<<grid, pa::kFwdThreads, pa::FwdCfg<128>::kSmemBytes, stream>>>(fp);
-  else
-    pa::attn_fwd_kernel<64><<<grid, pa::kFwdThreads, pa::FwdCfg<64>::kSmemBytes, stream>>>(fp);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  // Programmatic dependent launch: the attention kernel's prologue overlaps the
+  // schedule kernel, whose results it reads only after griddepcontrol.wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.dynamicSmemBytes = head_dim == 128 ? pa::FwdCfg<128>::kSmemBytes : pa::FwdCfg<64>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = g_prof_on ? 0 : 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = head_dim == 128 ? cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<128>, fp)
+                                         : cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<64>, fp);
+  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (g_prof_on) cudaEventRecord(ev1, stream);
   return PA_OK;
 }

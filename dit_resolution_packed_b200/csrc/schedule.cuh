@@ -86,6 +86,9 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   __shared__ int64_t s_total;
   const int tid = threadIdx.x;
   const int B = p.batch;
+  // the attention kernel may start its prologue now; it waits for this grid
+  // to complete before it reads anything written here
+  pdl_launch_dependents();
 
   if (tid == 0) s_bad = 0;
   for (int b = tid; b < kSortBuckets; b += kSchedThreads) s_hist[b] = 0;
