@@ -316,7 +316,8 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": f"bf16_tflops ({peak_src}, burst)",
                      "kernel": "attn_fwd_kernel<128>" if d == 128 else "attn_fwd_kernel<64>",
-                     "traffic": (trec or {}).get("dram_bytes_per_launch")},
+                     "traffic": (trec or {}).get("dram_bytes_per_launch"),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,  # schedule + attention kernel per step, headline timed region

@@ -90,14 +90,15 @@ struct Bars {
   uint64_t p_full[2][2];  // [tile][half]: P columns of keys 0-63 / 64-127 are in tensor memory
   uint64_t sched_full[2], sched_empty[2];  // work-item hand-off from the producer
   uint64_t drain;
-  int32_t sched_item[2];
+  int32_t sched_item[2][8];  // decoded items: seg, beg, len, head, q0, nkv, two, id; seg < 0 = done
   uint32_t tmem_base;
   int abort_flag;
 };
 
 struct WorkItem {
   int32_t seg, beg, len, head, q0, nkv;
-  bool two;  // second query tile has rows
+  bool two;    // second query tile has rows
+  int32_t id;  // index in the longest-first order
 };
 
 __device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p, int32_t n_sorted) {
@@ -116,6 +117,32 @@ __device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p
   w.q0 = (local - w.head * npairs) * 256;
   w.nkv = (w.len + 127) >> 7;
   w.two = w.q0 + 128 < w.len;
+  w.id = item;
+  return w;
+}
+
+// Work items travel decoded through the shared-memory ring: one global-memory
+// lookup per item by the producer instead of one per warp.
+__device__ __forceinline__ void store_item(volatile int32_t* d, const WorkItem& w) {
+  d[0] = w.seg;
+  d[1] = w.beg;
+  d[2] = w.len;
+  d[3] = w.head;
+  d[4] = w.q0;
+  d[5] = w.nkv;
+  d[6] = w.two ? 1 : 0;
+  d[7] = w.id;
+}
+__device__ __forceinline__ WorkItem load_item(const volatile int32_t* d) {
+  WorkItem w;
+  w.seg = d[0];
+  w.beg = d[1];
+  w.len = d[2];
+  w.head = d[3];
+  w.q0 = d[4];
+  w.nkv = d[5];
+  w.two = d[6] != 0;
+  w.id = d[7];
   return w;
 }
 
@@ -152,13 +179,17 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
     const uint32_t sph = (sk >> 1) & 1u;
     ++sk;
     if (!(ok = mbar_wait(&bars->sched_empty[ss], sph ^ 1u, wc))) break;
-    int32_t item = atomicAdd(p.next_item, 1);
-    if (item >= n_items) item = -1;
-    *reinterpret_cast<volatile int32_t*>(&bars->sched_item[ss]) = item;
+    const int32_t item = atomicAdd(p.next_item, 1);
+    WorkItem w;
+    if (item < n_items) {
+      w = decode_item(item, p, n_sorted);
+    } else {
+      w.seg = -1;
+    }
+    store_item(bars->sched_item[ss], w);
     mbar_arrive(&bars->sched_full[ss]);
-    if (item < 0) break;
+    if (w.seg < 0) break;
 
-    const WorkItem w = decode_item(item, p, n_sorted);
     const void* mq = seg_map(p, w.seg, 0);
     const void* mk = seg_map(p, w.seg, 1);
     const void* mv = seg_map(p, w.seg, 2);
@@ -207,16 +238,18 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
   }
 }
 
-// Takes the next item from the producer's hand-off ring; -1 when the work is done,
-// -2 when the wait gave up.  `arrive` releases the slot (one arrival per caller).
-__device__ __forceinline__ int32_t next_item_from_ring(Bars* bars, uint32_t& sk, const WaitCtl& wc, bool arrive) {
+// Takes the next decoded item from the producer's hand-off ring.  Returns 1 with
+// `w` filled, 0 when the work is done, -2 when the wait gave up.  `arrive`
+// releases the slot (one arrival per caller).
+__device__ __forceinline__ int next_item_from_ring(Bars* bars, uint32_t& sk, const WaitCtl& wc, bool arrive,
+                                                   WorkItem& w) {
   const int ss = sk & 1;
   const uint32_t sph = (sk >> 1) & 1u;
   ++sk;
   if (!mbar_wait(&bars->sched_full[ss], sph, wc)) return -2;
-  const int32_t item = *reinterpret_cast<volatile int32_t*>(&bars->sched_item[ss]);
+  w = load_item(bars->sched_item[ss]);
   if (arrive) mbar_arrive(&bars->sched_empty[ss]);
-  return item;
+  return w.seg < 0 ? 0 : 1;
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -262,10 +295,10 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
   uint32_t sk = 0;
   bool ok = true;
   for (;;) {
-    const int32_t item = next_item_from_ring(bars, sk, wc, true);
-    if (item == -2) ok = false;
-    if (item < 0) break;
-    const WorkItem w = decode_item(item, p, n_sorted);
+    WorkItem w;
+    const int got = next_item_from_ring(bars, sk, wc, true, w);
+    if (got == -2) ok = false;
+    if (got <= 0) break;
     if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
     ++q_round;
     int ks = slot;
@@ -432,13 +465,13 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
   bool ok = true;
 
   for (;;) {
-    int32_t item = next_item_from_ring(bars, sk, wc, false);
-    if (__any_sync(0xffffffffu, item == -2)) item = -2;
+    WorkItem w;
+    int got = next_item_from_ring(bars, sk, wc, false, w);
+    if (__any_sync(0xffffffffu, got == -2)) got = -2;
     __syncwarp();
-    if (lane == 0 && item != -2) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
-    if (item == -2) ok = false;
-    if (item < 0) break;
-    const WorkItem w = decode_item(item, p, n_sorted);
+    if (lane == 0 && got != -2) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
+    if (got == -2) ok = false;
+    if (got <= 0) break;
     if (tile == 1 && !w.two) continue;
     // l: sum of the fp32 exponentials (gives lse); lr: sum of the same values rounded to
     // bf16, i.e. of the weights the P.V product actually used (normalises the output,

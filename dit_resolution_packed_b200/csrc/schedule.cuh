@@ -1,6 +1,6 @@
 // schedule.cuh -- device-side segment scheduler for the packed attention kernel.
 //
-// One CTA of 1024 threads turns cu_seqlens into the work list of the attention
+// One CTA of 256 threads turns cu_seqlens into the work list of the attention
 // kernel, without a host round trip:
 //   1. validates cu_seqlens (cu[0] = 0, non-decreasing, cu[B] = T, every
 //      segment <= max_seqlen); on failure it records the status and publishes
@@ -28,8 +28,9 @@
 
 namespace pa {
 
-constexpr int kSchedThreads = 1024;
-constexpr int kSortBuckets = 4096;  // tile counts >= 4095 share the first bucket
+constexpr int kSchedThreads = 256;
+constexpr int kSortBuckets = 1024;     // tile counts >= 1023 share the first bucket
+constexpr int kCuInSmem = 4096 + 1;    // cu_seqlens staged in shared memory up to this many entries
 
 struct SchedParams {
   CUtensorMap tmpl[3];     // q, k, v over the whole [T, H*d] matrix (host-encoded)
@@ -50,8 +51,9 @@ __device__ __forceinline__ int seg_key(int32_t len) {
   return t < kSortBuckets - 1 ? t : kSortBuckets - 1;
 }
 
-// Exclusive prefix sum over the 1024 threads of the block; also returns the block total.
+// Exclusive prefix sum over the threads of the block; also returns the block total.
 __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* s_warp, int64_t* s_total) {
+  constexpr int kWarps = kSchedThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t x = v;
 #pragma unroll
@@ -62,13 +64,13 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* s_wa
   if (lane == 31) s_warp[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int64_t w = s_warp[lane], wx = w;
+    int64_t w = lane < kWarps ? s_warp[lane] : 0, wx = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int64_t y = __shfl_up_sync(0xffffffffu, wx, o);
       if (lane >= o) wx += y;
     }
-    s_warp[lane] = wx - w;
+    if (lane < kWarps) s_warp[lane] = wx - w;
     if (lane == 31) *s_total = wx;
   }
   __syncthreads();
@@ -79,6 +81,7 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* s_wa
 
 __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid_constant__ SchedParams p) {
   __shared__ int s_bad;
+  __shared__ int32_t s_cu_buf[kCuInSmem];
   __shared__ int32_t s_hist[kSortBuckets];
   __shared__ int32_t s_start[kSortBuckets];
   __shared__ int32_t s_keys[kSchedThreads];
@@ -90,14 +93,18 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   // to complete before it reads anything written here
   pdl_launch_dependents();
 
+  // cu_seqlens in shared memory (one pass over global memory) when it fits
+  const bool staged = B + 1 <= kCuInSmem;
+  for (int i = tid; staged && i <= B; i += kSchedThreads) s_cu_buf[i] = p.cu[i];
+  const int32_t* cu = staged ? s_cu_buf : p.cu;
   if (tid == 0) s_bad = 0;
   for (int b = tid; b < kSortBuckets; b += kSchedThreads) s_hist[b] = 0;
   __syncthreads();
 
   // 1. validation and histogram of tile counts
-  if (tid == 0 && (p.cu[0] != 0 || p.cu[B] != p.total)) atomicMax(&s_bad, 2);
+  if (tid == 0 && (cu[0] != 0 || cu[B] != p.total)) atomicMax(&s_bad, 2);
   for (int i = tid; i < B; i += kSchedThreads) {
-    const int32_t a = p.cu[i], b = p.cu[i + 1];
+    const int32_t a = cu[i], b = cu[i + 1];
     if (b < a) {
       atomicMax(&s_bad, 2);
     } else if (b - a > p.max_seqlen) {
@@ -117,7 +124,21 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     return;
   }
 
-  // 2. bucket offsets in descending tile-count order (each thread owns 4 buckets)
+  // 2. per-segment tensor maps: copy the template, then move its base and row extent
+  for (int idx = tid; idx < 3 * B; idx += kSchedThreads) {
+    const int s = idx / 3, which = idx - 3 * s;
+    const int32_t beg = cu[s], len = cu[s + 1] - beg;
+    if (len <= 0) continue;
+    uint8_t* dst = p.maps + static_cast<size_t>(idx) * 128;
+    const uint4* src = reinterpret_cast<const uint4*>(&p.tmpl[which]);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) reinterpret_cast<uint4*>(dst)[w] = src[w];
+    const uint8_t* seg_base = static_cast<const uint8_t*>(p.base[which]) + static_cast<uint64_t>(beg) * p.row_bytes;
+    tmap_replace_address(dst, seg_base);
+    tmap_replace_dim1(dst, static_cast<uint32_t>(len));
+  }
+
+  // 3. bucket offsets in descending tile-count order (each thread owns 4 buckets)
   {
     constexpr int per = kSortBuckets / kSchedThreads;
     int64_t local = 0;
@@ -135,12 +156,13 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   const int32_t n_sorted = static_cast<int32_t>(s_total);
   __syncthreads();
 
-  // Stable placement: within a bucket segments keep their packing order.
+  // 4. stable placement (within a bucket segments keep their packing order) and,
+  // in the same pass, the first work item of every ordered segment
   for (int c0 = 0; c0 < B; c0 += kSchedThreads) {
     const int i = c0 + tid;
     int key = -1;
     if (i < B) {
-      const int32_t len = p.cu[i + 1] - p.cu[i];
+      const int32_t len = cu[i + 1] - cu[i];
       if (len > 0) key = seg_key(len);
     }
     s_keys[tid] = key;
@@ -157,14 +179,13 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   __threadfence_block();
   __syncthreads();
 
-  // 3. first work item of every ordered segment
   int64_t carry = 0;
   for (int c0 = 0; c0 < n_sorted; c0 += kSchedThreads) {
     const int k = c0 + tid;
     int64_t items = 0;
     if (k < n_sorted) {
       const int s = p.order[k];
-      const int32_t len = p.cu[s + 1] - p.cu[s];
+      const int32_t len = cu[s + 1] - cu[s];
       items = static_cast<int64_t>(p.heads) * ((len + 255) >> 8);
     }
     const int64_t ex = block_exclusive_scan(items, s_warp, &s_total);
@@ -177,20 +198,6 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     p.counts[0] = static_cast<int32_t>(carry);
     p.counts[1] = n_sorted;
     p.counts[2] = 0;
-  }
-
-  // 4. per-segment tensor maps: copy the template, then move its base and row extent
-  for (int idx = tid; idx < 3 * B; idx += kSchedThreads) {
-    const int s = idx / 3, which = idx - 3 * s;
-    const int32_t beg = p.cu[s], len = p.cu[s + 1] - beg;
-    if (len <= 0) continue;
-    uint8_t* dst = p.maps + static_cast<size_t>(idx) * 128;
-    const uint4* src = reinterpret_cast<const uint4*>(&p.tmpl[which]);
-#pragma unroll
-    for (int w = 0; w < 8; ++w) reinterpret_cast<uint4*>(dst)[w] = src[w];
-    const uint8_t* seg_base = static_cast<const uint8_t*>(p.base[which]) + static_cast<uint64_t>(beg) * p.row_bytes;
-    tmap_replace_address(dst, seg_base);
-    tmap_replace_dim1(dst, static_cast<uint32_t>(len));
   }
   fence_tmap_release();
 }
