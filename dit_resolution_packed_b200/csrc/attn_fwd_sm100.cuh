@@ -60,11 +60,21 @@ struct FwdCfg {
   static constexpr int kSlots = (D == 128) ? 5 : 10;     // K/V ring depth (tiles)
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
+  // d = 64: V is extended by a tile of bf16 ones (one 64-column swizzle atom, shared
+  // by all slots), so the P.V product also yields sum_k bf16(P) in O's column d:
+  // the exact normaliser of the output, computed by the tensor core.
+  static constexpr bool kSumColumn = (D == 64);
+  static constexpr int kOCols = kSumColumn ? D + 16 : D;  // O columns written by P.V
+  static constexpr int kOffOnes = kOffKV + kSlots * kTileBytes;
+  static constexpr int kOffBar = kOffOnes + (kSumColumn ? kRows * 128 : 0);
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // + 1024 for base alignment
   static constexpr uint32_t kTmemCols = 512;
-  __host__ __device__ static constexpr uint32_t col_s(int tile) { return tile ? 128u : 0u; }
-  __host__ __device__ static constexpr uint32_t col_o(int tile) { return tile ? 256u + D : 256u; }
+  // tensor memory: d = 128: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
+  //                d = 64:  S0 [0,128) O0 [128,208) S1 [256,384) O1 [384,464)
+  __host__ __device__ static constexpr uint32_t col_s(int tile) { return kSumColumn ? (tile ? 256u : 0u) : (tile ? 128u : 0u); }
+  __host__ __device__ static constexpr uint32_t col_o(int tile) {
+    return kSumColumn ? (tile ? 384u : 128u) : (tile ? 256u + D : 256u);
+  }
 };
 
 struct FwdParams {
@@ -268,13 +278,17 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32
   }
 }
 
-// O (+)= P V over the keys [64*half, 64*half + 64) of the tile.
+// O (+)= P V over the keys [64*half, 64*half + 64) of the tile.  With a sum
+// column, V's second 64-column swizzle atom is the shared tile of ones: the
+// descriptor's leading byte offset points from the V slot to it.
 template <int D>
-__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, int half,
-                                              bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, uint32_t ones_addr,
+                                              int half, bool accumulate) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16_f32(128, C::kOCols, true);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
-  const uint32_t b0 = sdesc_sw128_lo(v_addr, FwdCfg<D>::kBlockBytes);
+  const uint32_t lbo = C::kSumColumn ? ones_addr - v_addr : C::kBlockBytes;
+  const uint32_t b0 = sdesc_sw128_lo(v_addr, lbo);
 #pragma unroll
   for (int kq = 0; kq < 4; ++kq) {
     const int kk = half * 4 + kq;
@@ -289,6 +303,7 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
   using C = FwdCfg<D>;
   const uint32_t q_addr0 = smem_u32(smem + C::kOffQ);
   const uint32_t kv_addr0 = smem_u32(smem + C::kOffKV);
+  const uint32_t ones_addr = smem_u32(smem + C::kOffOnes);
   int slot = 0;
   uint32_t phase = 0, q_round = 0;
   uint32_t p_ph = 0, oe_ph = 0;  // bit t: phase of tile t
@@ -327,11 +342,11 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
         }
         if (!(ok = mbar_wait(&bars->p_full[t][0], (p_ph >> t) & 1u, wc))) break;
         tc_fence_after();
-        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, 0, j > 0);
+        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 0, j > 0);
         if (!(ok = mbar_wait(&bars->p_full[t][1], (p_ph >> t) & 1u, wc))) break;
         p_ph ^= 1u << t;
         tc_fence_after();
-        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, 1, true);
+        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 1, true);
         if (has_next) {
           if (t == 0) {  // K_{j+1} is needed only now, after P.V of tile 0 is queued
             ks = slot;
@@ -405,8 +420,9 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
     lr *= alpha;
     m = m_new;
     // O += P V of the previous tile has completed (S of this tile was issued after it).
+    // With a sum column, the rescale covers it too (it accumulates like O).
 #pragma unroll
-    for (int cc = 0; cc < D / 16; ++cc) {
+    for (int cc = 0; cc < FwdCfg<D>::kOCols / 16; ++cc) {
       uint32_t o[16];
       PA_TMEM_LD16(tO + cc * 16, o);
       tmem_wait_ld();
@@ -436,7 +452,7 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
         const uint64_t pp = (!kPartial && (k & 3) >= 4 - kPolyPairsPer4) ? ex2x2_poly(x, ek) : ex2x2(x);
         const uint32_t pr = pack_bf16x2_pair(pp);
         su[k & 1] = f2_add(su[k & 1], pp);
-        sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
+        if (!FwdCfg<D>::kSumColumn) sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
         pk[k] = pr;
       }
       PA_TMEM_ST16(tS + cc * 16, pk);
@@ -448,7 +464,7 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
   }
   const uint64_t su2 = f2_add(su[0], su[1]), sr2 = f2_add(sr[0], sr[1]);
   l += f2_lo(su2) + f2_hi(su2);
-  lr += f2_lo(sr2) + f2_hi(sr2);
+  if (!FwdCfg<D>::kSumColumn) lr += f2_lo(sr2) + f2_hi(sr2);
 }
 
 template <int D>
@@ -506,6 +522,13 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
     const bool row_ok = row < w.len;
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
                                           (static_cast<size_t>(w.beg + (row_ok ? row : 0)) * p.heads + w.head) * D);
+    if (C::kSumColumn) {
+      // sum of the bf16 weights, accumulated by the tensor core in O's column d
+      uint32_t sc[16];
+      PA_TMEM_LD16(tO + D, sc);
+      tmem_wait_ld();
+      lr = __uint_as_float(sc[0]);
+    }
     const float inv_l = 1.0f / lr;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -559,6 +582,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
+  }
+  if (C::kSumColumn) {
+    // the tile of ones read by P.V as V's extra columns (bf16 1.0 = 0x3F80)
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::kOffOnes);
+    for (int i = threadIdx.x; i < C::kRows * 128 / 16; i += kFwdThreads)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    fence_proxy_async_smem();  // visible to the tensor core (async proxy)
   }
   if (warp == 9) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
