@@ -29,6 +29,8 @@ PA_ERR_TIMEOUT = -7
 PA_ERR_CUDA = -8
 PA_ERR_SCALE = -9
 PA_ERR_NOT_DEVICE = -10
+PA_ERR_NOALLOC_LIMIT = -11
+NOALLOC_MAX_BATCH = 1024
 
 _lib = None
 
@@ -52,6 +54,9 @@ def load_library(path=None):
     vp, i32 = ctypes.c_void_p, ctypes.c_int32
     lib.pa_varlen_attn_fwd.restype = ctypes.c_int
     lib.pa_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp]
+    lib.pa_varlen_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.pa_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp,
+                                               vp, vp]
     lib.pa_get_error.restype = ctypes.c_int
     lib.pa_get_error.argtypes = [vp]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -109,6 +114,35 @@ def pa_varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale, out, lse, stream=
     return load_library().pa_varlen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, T, H, d,
                                              int(max_seqlen), float(scale), _ptr(out), _ptr(lse),
                                              _stream_handle(stream))
+
+
+def pa_varlen_attn_fwd_noalloc(q, k, v, cu_seqlens, max_seqlen, scale, out, lse, status=None, stream=None):
+    """C ``pa_varlen_attn_fwd_noalloc``: the forward without any device allocation by the library.
+
+    For callers whose device memory is owned by someone else (a framework's
+    caching allocator or arena, a plug-in host, a serving loop that must not
+    allocate): every buffer is the caller's -- q, k, v, out bf16 [T, H, d],
+    cu_seqlens int32 [B+1], lse fp32 [T, H], and optionally ``status``, an int32
+    device tensor of at least one element that receives this call's device-side
+    error code.  The library's own scratch is a fixed array in its device image
+    (at most ``NOALLOC_MAX_BATCH`` segments); calls that overlap on one GPU race
+    on it.  Returns the host-side status code."""
+    import torch
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("out", out, torch.bfloat16), ("cu_seqlens", cu_seqlens, torch.int32),
+                        ("lse", lse, torch.float32)) + ((("status", status, torch.int32),) if status is not None
+                                                        else ()):
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    T, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or out.shape != q.shape or tuple(lse.shape) != (T, H):
+        raise ValueError("shape mismatch: q, k, v, out [T, H, d]; lse [T, H]")
+    B = cu_seqlens.numel() - 1
+    return load_library().pa_varlen_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, T, H, d,
+                                                     int(max_seqlen), float(scale), _ptr(out), _ptr(lse),
+                                                     _ptr(status), _stream_handle(stream))
 
 
 def varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale=None, out=None, lse=None, stream=None):

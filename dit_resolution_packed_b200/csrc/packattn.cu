@@ -148,6 +148,38 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 }  // namespace
 
+// ---- scratch of pa_varlen_attn_fwd_noalloc ----------------------------------
+// One fixed array in the library's device image: the status word (bytes
+// [0, 256)) and, from byte 256, the schedule + per-segment tensor maps laid out
+// as in the allocating path.  Every GPU that loads the library holds it until
+// the process exits; every call on that GPU shares it.
+constexpr int32_t kNoAllocMaxBatch = 1024;
+constexpr size_t kNoAllocStatusBytes = 256;
+constexpr size_t kNoAllocScratchBytes = 400 * 1024;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch per device (the host-side name is only a
+// stand-in for the symbol); filled by the first call on each device.
+uint8_t* g_noalloc_ptr[64] = {};
+
+// The device must be current; g_mu held.
+int noalloc_setup(int device) {
+  if (g_noalloc_ptr[device]) return PA_OK;
+  if (kNoAllocStatusBytes + ws_layout(kNoAllocMaxBatch).total > kNoAllocScratchBytes) return PA_ERR_CUDA;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  if (!p || !aligned(p, 256)) return PA_ERR_CUDA;
+  g_noalloc_ptr[device] = static_cast<uint8_t*>(p);
+  return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
@@ -291,6 +323,7 @@ const char* pa_status_string(int code) {
     case PA_ERR_CUDA: return "CUDA runtime error";
     case PA_ERR_SCALE: return "scale is not finite";
     case PA_ERR_NOT_DEVICE: return "a buffer is not device memory of one GPU";
+    case PA_ERR_NOALLOC_LIMIT: return "batch exceeds the 1024 segments of pa_varlen_attn_fwd_noalloc's fixed scratch";
     default: return "unknown status";
   }
 }
@@ -349,6 +382,103 @@ int pa_profile_read(double* total_ms, int32_t* launches) {
   if (total_ms) *total_ms = sum;
   if (launches) *launches = static_cast<int32_t>(g_prof_used);
   g_prof_used = 0;
+  return PA_OK;
+}
+
+int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                               int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim,
+                               int32_t max_seqlen, float scale, void* out, float* lse, int32_t* status,
+                               void* stream_handle) {
+  // ---- host-visible argument checks: nothing is enqueued on failure
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
+  if (batch > kNoAllocMaxBatch) return PA_ERR_NOALLOC_LIMIT;
+  if (!std::isfinite(scale)) return PA_ERR_SCALE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  if (max_seqlen < 1) return PA_ERR_MAX_SEQLEN;
+  if (!q || !k || !v || !cu_seqlens || !out || !lse) return PA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+      !aligned(cu_seqlens, 4) || (status && !aligned(status, 4)))
+    return PA_ERR_ALIGN;
+  const int64_t item_bound = static_cast<int64_t>(heads) * ((static_cast<int64_t>(total_tokens) + 255) / 256 + batch);
+  if (item_bound >= (int64_t(1) << 31) || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24))
+    return PA_ERR_SHAPE;
+
+  int dev = -1, d2 = -1;
+  int rc;
+  if ((rc = device_of(q, &dev)) != PA_OK) return rc;
+  const void* others[6] = {k, v, out, lse, cu_seqlens, status};
+  for (const void* p : others) {
+    if (!p) continue;  // only status may be NULL here
+    if ((rc = device_of(p, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  if ((rc = noalloc_setup(dev)) != PA_OK) return rc;
+  uint8_t* scratch = g_noalloc_ptr[dev];
+  uint8_t* ws = scratch + kNoAllocStatusBytes;
+  int32_t* st = status ? status : reinterpret_cast<int32_t*>(scratch);
+  const WsLayout L = ws_layout(batch);
+
+  // The status word must start at zero; the schedule kernel rewrites the rest
+  // (counts, work counter, order, item starts, tensor maps) before it is read.
+  if (cudaMemsetAsync(st, 0, sizeof(int32_t), stream) != cudaSuccess) return PA_ERR_CUDA;
+
+  pa::SchedParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  const void* bases[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
+    sp.base[i] = bases[i];
+  }
+  sp.cu = cu_seqlens;
+  sp.status = st;
+  sp.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  sp.order = reinterpret_cast<int32_t*>(ws + L.order);
+  sp.item_start = reinterpret_cast<int32_t*>(ws + L.item_start);
+  sp.maps = ws + L.maps;
+  sp.row_bytes = static_cast<uint64_t>(heads) * head_dim * 2;
+  sp.batch = batch;
+  sp.total = total_tokens;
+  sp.heads = heads;
+  sp.max_seqlen = max_seqlen;
+  sp.err_cu = PA_ERR_CU_SEQLENS;
+  sp.err_max = PA_ERR_MAX_SEQLEN;
+  pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  pa::FwdParams fp;
+  fp.cu = cu_seqlens;
+  fp.out = out;
+  fp.lse = lse;
+  fp.counts = sp.counts;
+  fp.next_item = sp.counts + 2;
+  fp.order = sp.order;
+  fp.item_start = sp.item_start;
+  fp.maps = sp.maps;
+  fp.status = st;
+  fp.heads = heads;
+  fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  fp.err_timeout = PA_ERR_TIMEOUT;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound)));
+  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.dynamicSmemBytes = head_dim == 128 ? pa::FwdCfg<128>::kSmemBytes : pa::FwdCfg<64>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = head_dim == 128 ? cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<128>, fp)
+                                         : cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<64>, fp);
+  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 

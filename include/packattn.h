@@ -44,7 +44,8 @@ enum pa_status {
   PA_ERR_TIMEOUT = -7,      /* device: a pipeline wait exceeded its limit; the kernel stopped early */
   PA_ERR_CUDA = -8,         /* a CUDA runtime call or a kernel launch failed */
   PA_ERR_SCALE = -9,        /* scale is not finite */
-  PA_ERR_NOT_DEVICE = -10   /* q, k, v, out, lse or cu_seqlens is not device memory of one GPU */
+  PA_ERR_NOT_DEVICE = -10,  /* q, k, v, out, lse or cu_seqlens is not device memory of one GPU */
+  PA_ERR_NOALLOC_LIMIT = -11 /* pa_varlen_attn_fwd_noalloc: batch above its 1024-segment maximum */
 };
 
 /*
@@ -128,6 +129,52 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
  */
 PA_API void pa_profile_enable(int on);
 PA_API int pa_profile_read(double* total_ms, int32_t* launches);
+
+/*
+ * pa_varlen_attn_fwd_noalloc -- the same forward as pa_varlen_attn_fwd (same
+ * kernels, same results bit for bit), for callers that must not allocate
+ * device memory.  None of the pages defines this entry point: it is a service
+ * of this library and has no counterpart in the method.
+ *
+ * Who needs it: code whose device memory belongs to someone else -- a framework
+ * whose caching allocator or pre-reserved arena owns nearly all of the GPU (a
+ * cudaMalloc there fails or fragments memory the owner cannot see), a plug-in
+ * whose enqueue is called in a context that forbids allocation, or a serving
+ * loop that must not allocate after warm-up.  Such a caller already owns q, k,
+ * v, cu_seqlens, out and lse; the one thing pa_varlen_attn_fwd adds is its own
+ * workspace (schedule, per-segment tensor maps, status word), grown with
+ * cudaMallocAsync.  This entry point uses instead a fixed 400 KiB array that is
+ * part of the library's device image: every GPU that loads the library holds it
+ * until the process exits.  The call allocates nothing (no cudaMalloc,
+ * cudaMallocAsync, cudaFree or allocating library routine).
+ *
+ *   Arguments q ... lse and stream: as for pa_varlen_attn_fwd.
+ *   batch        at most 1024 segments; a larger batch returns
+ *                PA_ERR_NOALLOC_LIMIT and enqueues nothing.
+ *   status       optional device int32 (4-byte aligned, same GPU).  The call
+ *                sets it to 0 on `stream`, and the kernels record there a
+ *                device-side error (PA_ERR_CU_SEQLENS, PA_ERR_MAX_SEQLEN,
+ *                PA_ERR_TIMEOUT) of this call; read it after the stream has
+ *                finished.  With NULL a status word inside the fixed array is
+ *                used (cleared by each call) and such errors are not reported.
+ *                pa_get_error does not see this entry point's errors.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and sets the kernels'
+ * shared-memory attributes; that first call may also make the CUDA runtime load
+ * the library's kernels onto the device.  Make it before any stream capture.
+ *
+ * Sharing: all calls on one GPU use the same array, which keeps the contents of
+ * the last call; each call clears the status word and rewrites everything else
+ * before reading it.  Calls whose work overlaps on that GPU (different streams,
+ * or different host threads without ordering between their streams) race on
+ * the array and give undefined results: order them on one stream or with
+ * events.  Host-side use is thread-safe.
+ */
+PA_API int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                      int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                      int32_t max_seqlen, float scale, void* out, float* lse, int32_t* status,
+                                      void* stream);
 
 #ifdef __cplusplus
 }

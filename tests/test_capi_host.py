@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 9
+    assert len(names) == len(set(names)) == 10
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert pa.pa_version() == 100
-    codes = [0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10]
+    codes = [0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -11]
     texts = [pa.status_string(c) for c in codes]
     assert len(set(texts)) == len(codes) and "unknown" not in " ".join(texts)
     assert pa.status_string(-99) == "unknown status"
@@ -65,6 +65,16 @@ def test_host_validation_before_any_cuda_call(lib):
     assert _raw(lib, out=8) == pa.PA_ERR_ALIGN
     assert _raw(lib, lse=18) == pa.PA_ERR_ALIGN
     assert _raw(lib, heads=1 << 20, head_dim=64, total=1 << 30) == pa.PA_ERR_SHAPE
+
+
+def test_noalloc_rejects_batch_above_its_limit_before_any_cuda_call(lib):
+    f = lib.pa_varlen_attn_fwd_noalloc
+    args = lambda batch, head_dim=64: (16, 16, 16, 16, batch, 4096, 1, head_dim, 4, ctypes.c_float(0.125), 16, 16,
+                                       None, None)
+    assert f(*args(pa.NOALLOC_MAX_BATCH + 1)) == pa.PA_ERR_NOALLOC_LIMIT
+    assert f(*args(1 << 30)) == pa.PA_ERR_NOALLOC_LIMIT
+    assert f(*args(pa.NOALLOC_MAX_BATCH, head_dim=96)) == pa.PA_ERR_HEAD_DIM
+    assert f(16, 16, 16, 16, 3, 0, 1, 64, 4, ctypes.c_float(0.125), 16, 16, None, None) == pa.PA_OK
 
 
 def test_missing_library_fails_loudly(tmp_path):
