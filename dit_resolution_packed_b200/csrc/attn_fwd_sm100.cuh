@@ -267,14 +267,14 @@ __device__ __forceinline__ int next_item_from_ring(Bars* bars, uint32_t& sk, con
 // addresses change (no carry leaves the 14-bit field: shared-memory addresses
 // are below 256 KB), the high word is one constant.
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_s(uint32_t issue, uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
   const uint32_t a0 = sdesc_sw128_lo(q_addr, 16), b0 = sdesc_sw128_lo(k_addr, 16);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = ((kk >> 2) * FwdCfg<D>::kBlockBytes + (kk & 3) * 32) >> 4;
-    mma_bf16_ss_lo(d_tmem, a0 + off, b0 + off, hi, idesc, kk > 0 ? 1u : 0u);
+    mma_bf16_ss_lo_if(issue, d_tmem, a0 + off, b0 + off, hi, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -282,8 +282,8 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32
 // column, V's second 64-column swizzle atom is the shared tile of ones: the
 // descriptor's leading byte offset points from the V slot to it.
 template <int D>
-__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, uint32_t ones_addr,
-                                              int half, bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(uint32_t issue, uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                              uint32_t ones_addr, int half, bool accumulate) {
   using C = FwdCfg<D>;
   constexpr uint32_t idesc = idesc_bf16_f32(128, C::kOCols, true);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
@@ -292,7 +292,7 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
 #pragma unroll
   for (int kq = 0; kq < 4; ++kq) {
     const int kk = half * 4 + kq;
-    mma_bf16_ts_lo(d_tmem, p_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
+    mma_bf16_ts_lo_if(issue, d_tmem, p_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
                    (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -309,9 +309,11 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
   uint32_t p_ph = 0, oe_ph = 0;  // bit t: phase of tile t
   uint32_t sk = 0;
   bool ok = true;
+  const uint32_t leader = elect_one_sync();
   for (;;) {
     WorkItem w;
-    const int got = next_item_from_ring(bars, sk, wc, true, w);
+    const int got = next_item_from_ring(bars, sk, wc, false, w);
+    if (got != -2 && leader) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
     if (got == -2) ok = false;
     if (got <= 0) break;
     if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
@@ -323,11 +325,11 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if (t == 1 && !w.two) break;
-      issue_s<D>(tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
-      mma_commit(&bars->s_full[t]);
+      issue_s<D>(leader, tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
+      mma_commit_if(leader, &bars->s_full[t]);
     }
-    mma_commit(&bars->kv_empty[ks]);
-    if (w.nkv == 1) mma_commit(&bars->q_empty);
+    mma_commit_if(leader, &bars->kv_empty[ks]);
+    if (w.nkv == 1) mma_commit_if(leader, &bars->q_empty);
     for (int32_t j = 0; ok && j < w.nkv; ++j) {
       const bool has_next = j + 1 < w.nkv;
       const int vs = slot;
@@ -342,11 +344,11 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
         }
         if (!(ok = mbar_wait(&bars->p_full[t][0], (p_ph >> t) & 1u, wc))) break;
         tc_fence_after();
-        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 0, j > 0);
+        issue_pv_half<D>(leader, tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 0, j > 0);
         if (!(ok = mbar_wait(&bars->p_full[t][1], (p_ph >> t) & 1u, wc))) break;
         p_ph ^= 1u << t;
         tc_fence_after();
-        issue_pv_half<D>(tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 1, true);
+        issue_pv_half<D>(leader, tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 1, true);
         if (has_next) {
           if (t == 0) {  // K_{j+1} is needed only now, after P.V of tile 0 is queued
             ks = slot;
@@ -354,23 +356,23 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
             if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
             tc_fence_after();
           }
-          issue_s<D>(tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
-          mma_commit(&bars->s_full[t]);
+          issue_s<D>(leader, tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
+          mma_commit_if(leader, &bars->s_full[t]);
         } else {
-          mma_commit(&bars->o_full[t]);
+          mma_commit_if(leader, &bars->o_full[t]);
         }
       }
       if (!ok) break;
-      mma_commit(&bars->kv_empty[vs]);
+      mma_commit_if(leader, &bars->kv_empty[vs]);
       if (has_next) {
-        mma_commit(&bars->kv_empty[ks]);
-        if (j + 2 == w.nkv) mma_commit(&bars->q_empty);
+        mma_commit_if(leader, &bars->kv_empty[ks]);
+        if (j + 2 == w.nkv) mma_commit_if(leader, &bars->q_empty);
       }
     }
     if (!ok) break;
   }
   // Every MMA issued so far completes before tensor memory is released.
-  mma_commit(&bars->drain);
+  mma_commit_if(leader, &bars->drain);
   drain_wait(&bars->drain, 0, wc.limit_ns);
 }
 
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     if (warp == 8) {
       if ((threadIdx.x & 31) == 0) run_producer<D>(p, smem, bars, wc, n_items, n_sorted);
     } else if (warp == 9) {
-      if ((threadIdx.x & 31) == 0) run_mma<D>(p, smem, bars, wc, tmem, n_sorted);
+      run_mma<D>(p, smem, bars, wc, tmem, n_sorted);  // the whole warp; one elected lane issues
     }
     __syncwarp();
     tc_fence_before();
