@@ -19,7 +19,9 @@
 //   warps 0-3  softmax + epilogue of query tile 0 (one thread per row)
 //   warps 4-7  softmax + epilogue of query tile 1
 //   warp 8     TMA producer: Q tiles, then K_j, V_j into a ring of smem slots
-//   warp 9     tensor-memory owner and MMA issuer
+//   warp 9     tensor-memory owner and MMA issuer (the whole warp runs the issue
+//              loop so its operand arithmetic stays warp-uniform; one elected
+//              lane issues the MMAs and commits)
 //   warps 10-11 idle (they complete the third warpgroup for the register split)
 // Tensor memory (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1.  P (bf16)
 // overwrites the first half of its S columns and feeds the P.V MMA from tensor
@@ -34,16 +36,20 @@
 
 namespace pa {
 
-constexpr float kRescaleLog2 = 8.0f;
-// In every group of four key pairs of a full score tile, this many are
-// exponentiated on the FMA pipe (polynomial) instead of the MUFU unit.
-// Measured on B200: 1 of 4 costs 8-10 % at d = 128 (issue slots, not MUFU,
-// bound this softmax), so it is off.
-constexpr int kPolyPairsPer4 = 0;
+// P <= 2^12 between moves of the shift: exact in bf16's exponent range, and O, l
+// stay far from fp32 overflow.  Measured on B200: 12 instead of 8 saves ~2 % on a
+// single 16384-token segment (fewer O rescales), nothing elsewhere.
+constexpr float kRescaleLog2 = 12.0f;
+// In every group of four key pairs of a full score tile at head_dim 128, this many
+// are exponentiated on the FMA pipe (polynomial, max relative error below 1e-4,
+// far under the bf16 rounding of P) instead of the MUFU unit.  Measured on B200
+// with the warp-wide MMA issuer: 1 of 4 gains ~2 % at d = 128; at d = 64 it loses
+// ~1 %, and 2 of 4 spills registers.
+constexpr int kPolyPairsPer4 = 1;
 constexpr int kFwdThreads = 384;
 // Register split of the 384-thread block launched at 168 registers per thread
-// (384 x 168 = 64512): the two softmax warpgroups rise to 224, the producer /
-// MMA warpgroup drops to 56.  2*128*224 + 128*56 = 64512.  The build checks
+// (384 x 168 = 64512): the two softmax warpgroups rise to 216, the producer /
+// MMA warpgroup drops to 72.  2*128*216 + 128*72 = 64512.  The build checks
 // that the kernels are compiled at exactly kLaunchRegs.
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 216;
@@ -413,25 +419,17 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
                                              uint32_t tS, uint32_t tO, float& m, float& l, float& lr,
                                              uint64_t* p_full_half, int lane) {
   const float xmax = row_extreme<kPartial, kNeg>(v, kv_valid) * c;  // log2 units
+  bool rescale = false;  // warp-uniform
+  float alpha = 1.f;
   if (first) {
     m = xmax;
   } else if (__any_sync(0xffffffffu, xmax > m + kRescaleLog2)) {
     const float m_new = fmaxf(m, xmax);
-    const float alpha = ex2_approx(m - m_new);
+    alpha = ex2_approx(m - m_new);
     l *= alpha;
     lr *= alpha;
     m = m_new;
-    // O += P V of the previous tile has completed (S of this tile was issued after it).
-    // With a sum column, the rescale covers it too (it accumulates like O).
-#pragma unroll
-    for (int cc = 0; cc < FwdCfg<D>::kOCols / 16; ++cc) {
-      uint32_t o[16];
-      PA_TMEM_LD16(tO + cc * 16, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-      PA_TMEM_ST16(tO + cc * 16, o);
-    }
+    rescale = true;
   }
   const uint64_t c2 = f2_pack(c, c);
   const uint64_t negm2 = f2_pack(-m, -m);
@@ -451,7 +449,8 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
         if (kPartial) {
           x = f2_pack(2 * i < kv_valid ? f2_lo(x) : -INFINITY, 2 * i + 1 < kv_valid ? f2_hi(x) : -INFINITY);
         }
-        const uint64_t pp = (!kPartial && (k & 3) >= 4 - kPolyPairsPer4) ? ex2x2_poly(x, ek) : ex2x2(x);
+        const uint64_t pp =
+            (!kPartial && D == 128 && (k & 3) >= 4 - kPolyPairsPer4) ? ex2x2_poly(x, ek) : ex2x2(x);
         const uint32_t pr = pack_bf16x2_pair(pp);
         su[k & 1] = f2_add(su[k & 1], pp);
         if (!FwdCfg<D>::kSumColumn) sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
@@ -459,10 +458,29 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
       }
       PA_TMEM_ST16(tS + cc * 16, pk);
     }
+    if (half == 1 && rescale) {
+      // O *= alpha, done after the exponentials, when the score registers are dead (with
+      // all 128 live, this block forced a spill whose reloads sat in the hot loop).  P.V
+      // of this tile has not started (half 0 is handed over only below, in rescale
+      // tiles) and that of the previous tile has completed (S of this tile was issued
+      // after it).  With a sum column, the rescale covers it too.
+#pragma unroll
+      for (int cc = 0; cc < FwdCfg<D>::kOCols / 16; ++cc) {
+        uint32_t o[16];
+        PA_TMEM_LD16(tO + cc * 16, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+        PA_TMEM_ST16(tO + cc * 16, o);
+      }
+    }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&p_full_half[half]);
+    if (lane == 0) {
+      if (half == 1 && rescale) mbar_arrive(&p_full_half[0]);
+      if (half == 1 || !rescale) mbar_arrive(&p_full_half[half]);
+    }
   }
   const uint64_t su2 = f2_add(su[0], su[1]), sr2 = f2_add(sr[0], sr[1]);
   l += f2_lo(su2) + f2_hi(su2);
@@ -561,7 +579,9 @@ template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived by an offset from the shared array (not through an
+  // integer round trip), so the compiler keeps every address below in the shared window.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
   const int warp = threadIdx.x >> 5;
 
