@@ -19,3 +19,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _library_matches_sources(request):
+    """GPU tests run against a library built from the current sources (rebuilt if older)."""
+    if any(item.get_closest_marker("gpu") for item in request.session.items):
+        from dit_resolution_packed_b200 import _build
+        _build.build()
