@@ -290,6 +290,7 @@ def run_ours(args, world, rank, local):
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, "timed region")
+    q10, q50, q90 = (float(x) for x in np.percentile(step_ms, [10, 50, 90]))
     total_ms = allreduce_max(sum(step_ms), world, device)
     ms_per_step = total_ms / args.steps
     value = flops * world / (ms_per_step * 1e-3) / 1e12
@@ -372,6 +373,10 @@ def run_ours(args, world, rank, local):
                        gpu_state="timed region follows the warm-up with no idle gap (power-limited steady state)",
                        parallelism=f"{world} independent replica(s), no collective"),
         "pct_of_bf16_peak": 100.0 * value / world / peak_burst,
+        "pct_of_bf16_sustained": 100.0 * value / world / float(
+            peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])),
+        "pct_of_bf16_datasheet_dense": 100.0 * value / world / 2250.0,  # vendor figure, not measured here
+        "step_ms_p10_p50_p90": [q10, q50, q90],
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "peak_source": (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_prof:.2f} s "

@@ -54,6 +54,15 @@ def test_many_short_segments_all_rows(cuda_device):
     _full_check(p, cuda_device)
 
 
+def test_batch_beyond_the_staged_schedule_path(cuda_device):
+    """5000 segments: more cu_seqlens entries than the scheduler stages in shared memory
+    (4097), so it reads them from global memory; short segments, all rows checked."""
+    rng = np.random.default_rng(8)
+    lens = rng.integers(0, 41, size=5000).tolist()
+    p = workloads.random_pack(lens, heads=2, head_dim=64, seed=22)
+    _full_check(p, cuda_device)
+
+
 def test_zero_length_segments(cuda_device):
     p = workloads.random_pack([0, 5, 0, 130, 0, 0, 257, 0], heads=2, head_dim=128, seed=13)
     _full_check(p, cuda_device)
