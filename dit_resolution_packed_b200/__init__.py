@@ -57,6 +57,9 @@ def load_library(path=None):
     lib.pa_varlen_attn_fwd_noalloc.restype = ctypes.c_int
     lib.pa_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp,
                                                vp, vp]
+    lib.pa_varlen_attn_bwd.restype = ctypes.c_int
+    lib.pa_varlen_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float,
+                                       vp, vp, vp, vp]
     lib.pa_get_error.restype = ctypes.c_int
     lib.pa_get_error.argtypes = [vp]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -158,6 +161,42 @@ def varlen_attn_fwd(q, k, v, cu_seqlens, max_seqlen, scale=None, out=None, lse=N
     if rc != PA_OK:
         raise PackAttnError(rc, "pa_varlen_attn_fwd")
     return out, lse
+
+
+def pa_varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, max_seqlen, scale, dq, dk, dv, stream=None):
+    """C ``pa_varlen_attn_bwd`` on torch tensors: q, k, v, out, dout, dq, dk, dv bf16 [T, H, d];
+    lse fp32 [T, H]; cu_seqlens int32 [B+1].  Returns the status code."""
+    import torch
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("out", out, torch.bfloat16), ("dout", dout, torch.bfloat16), ("dq", dq, torch.bfloat16),
+                        ("dk", dk, torch.bfloat16), ("dv", dv, torch.bfloat16), ("lse", lse, torch.float32),
+                        ("cu_seqlens", cu_seqlens, torch.int32)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    T, H, d = q.shape
+    for t in (k, v, out, dout, dq, dk, dv):
+        if t.shape != q.shape:
+            raise ValueError("shape mismatch: q, k, v, out, dout, dq, dk, dv [T, H, d]")
+    if tuple(lse.shape) != (T, H):
+        raise ValueError("lse must be [T, H]")
+    B = cu_seqlens.numel() - 1
+    return load_library().pa_varlen_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                             _ptr(cu_seqlens), B, T, H, d, int(max_seqlen), float(scale),
+                                             _ptr(dq), _ptr(dk), _ptr(dv), _stream_handle(stream))
+
+
+def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, max_seqlen, scale=None, stream=None):
+    """Gradients of ``varlen_attn_fwd``; returns (dq, dk, dv), bf16 [T, H, d]."""
+    import torch
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = pa_varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, max_seqlen, scale, dq, dk, dv, stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_varlen_attn_bwd")
+    return dq, dk, dv
 
 
 def pa_get_error(stream=None):

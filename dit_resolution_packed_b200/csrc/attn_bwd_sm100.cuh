@@ -1,0 +1,617 @@
+// attn_bwd_sm100.cuh -- gradients of the packed variable-length bidirectional
+// attention for B200 (sm_100a): dq, dk, dv from q, k, v, out, lse and dout.
+//
+// Math (chain rule through the row softmax of the forward definition; SparseAttn
+// page, section 3.1; GigaPath-Flash page, sections 3.2 / 4.2 for the blockwise
+// recomputation of P from the saved log-sum-exp): per segment, head, query row r
+// and key j of the segment,
+//     P_rj  = exp2(s_rj * scale * log2 e - lse_r * log2 e)     (recomputed)
+//     D_r   = dout_r . out_r                                    (prep kernel)
+//     dS_rj = scale * P_rj * (dout_r . v_j - D_r)
+//     dv_j += P_rj dout_r,   dk_j += dS_rj q_r,   dq_r += dS_rj k_j.
+//
+// Work item = (segment, head, 128-key tile): a persistent grid takes items
+// longest segment first (the scheduler kernel with 128-row items).  The CTA
+// keeps its K and V tiles in shared memory and dK, dV in tensor memory, and
+// walks the segment's 128-row query tiles; per query tile, five MMAs:
+//     S^T  = K Q^T        (A = K, B = Q, both K-major)        -> TMEM A
+//     dP^T = V dO^T       (A = V, B = dO, both K-major)       -> TMEM B
+//     dV  += P^T dO       (A = P^T bf16 in TMEM A, B = dO MN-major)
+//     dK  += dS^T Q       (A = dS^T bf16 in TMEM B, B = Q MN-major)
+//     dQ   = dS K         (A = dS^T in shared memory, read MN-major; B = K MN-major) -> TMEM B
+// and the next tile's S^T is issued between dK and dQ.  The dQ partial of every
+// (key tile, query tile) is added into an fp32 accumulator laid out [H][d/4][T]
+// (float4 per element group, token fastest), so that the 32 reductions of a warp
+// cover 512 contiguous bytes; a last kernel converts it to bf16 [T, H, d].
+//
+// Rows past the segment end are loaded (one tensor map per tensor over the whole
+// [T, H*d] matrix; past T the load reads zeros) and masked: a query past the
+// end has lse = +inf (so P = 0) and D = 0; a key past the end gets P = dS = 0.
+//
+// CTA layout, 12 warps:
+//   warps 0-3  elementwise: P^T and dS^T of one query tile (one thread per key row)
+//   warps 4-7  dQ partial -> fp32 reductions (one thread per query row); dK, dV
+//              epilogue at the end of the item (one thread per key row)
+//   warp 8     TMA producer (K, V once per item; Q, dO through a two-slot ring)
+//   warp 9     tensor-memory owner and MMA issuer (whole warp, one elected lane issues)
+//   warps 10-11 idle (they complete the third warpgroup for the register split)
+#pragma once
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace pa {
+
+constexpr int kBwdThreads = 384;
+constexpr int kBwdLaunchRegs = 168;
+constexpr int kBwdMathRegs = 216;
+constexpr int kBwdControlRegs = 72;
+static_assert(2 * 128 * kBwdMathRegs + 128 * kBwdControlRegs <= kBwdThreads * kBwdLaunchRegs, "register split");
+
+template <int D>
+struct BwdCfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int kRows = 128;
+  static constexpr int kTileBytes = kRows * D * 2;      // bf16 tile of 128 rows
+  static constexpr int kColBlocks = D / 64;             // 128-byte swizzle blocks across d
+  static constexpr int kBlockBytes = kRows * 128;       // one 64-column block of a tile
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;      // two ring slots
+  static constexpr int kOffDO = kOffQ + 2 * kTileBytes;  // two ring slots
+  static constexpr int kOffDS = kOffDO + 2 * kTileBytes;  // dS^T: 128 keys x 128 queries bf16, 2 blocks
+  static constexpr int kOffStage = kOffDS + 2 * kBlockBytes;  // -lse2 and -D*scale of the 128 queries
+  static constexpr int kOffBar = kOffStage + 2 * 128 * 4;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + 1024 for base alignment
+  static constexpr uint32_t kTmemCols = 512;
+  // tensor memory: A [0,128) S^T then P^T; B [128,256) dP^T, dS^T, then dQ;
+  // dV [256, 256+d); dK [256+d, 256+2d)
+  static constexpr uint32_t kColA = 0, kColB = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // [T, H*d] bf16, box {64, 128}, 128-byte swizzle
+  const int32_t* cu;
+  const int32_t* counts;     // [0] items, [1] ordered segments
+  int32_t* next_item;        // work counter, zeroed by the scheduler kernel
+  const int32_t* order;
+  const int32_t* item_start;
+  const float* lse2;         // [H][T] lse * log2(e)
+  const float* delta;        // [H][T] D = dout . out
+  float* dq_acc;             // [H][d/4][T] x 4 fp32
+  void* dk;                  // bf16 [T, H, d]
+  void* dv;                  // bf16 [T, H, d]
+  int32_t* status;
+  int32_t heads, total;
+  float scale, scale_log2;
+  uint64_t wait_limit_ns;
+  int32_t err_timeout;
+};
+
+struct BwdBars {
+  uint64_t kv_full, kv_empty;
+  uint64_t qd_full[2], qd_empty[2];
+  uint64_t s_full;     // S^T and dP^T of the current query tile are in tensor memory
+  uint64_t pds_full;   // P^T, dS^T stored (tensor memory and shared memory)
+  uint64_t dq_full, dq_empty;
+  uint64_t dkv_full, dkv_empty;
+  uint64_t stage_full, stage_empty;  // the per-query -lse2, -D*scale staging of the elementwise warps
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t drain;
+  int32_t sched_item[2][8];  // seg, beg, len, head, k0, n query tiles, -, id; seg < 0 = done
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(BwdBars) <= 256, "backward barrier block");
+
+struct BwdItem {
+  int32_t seg, beg, len, head, k0, nq, id;
+};
+
+__device__ __forceinline__ BwdItem bwd_decode_item(int32_t item, const BwdParams& p, int32_t n_sorted) {
+  int32_t lo = 0, hi = n_sorted;
+  while (hi - lo > 1) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (__ldg(p.item_start + mid) <= item) lo = mid; else hi = mid;
+  }
+  BwdItem w;
+  w.seg = __ldg(p.order + lo);
+  const int32_t local = item - __ldg(p.item_start + lo);
+  w.beg = __ldg(p.cu + w.seg);
+  w.len = __ldg(p.cu + w.seg + 1) - w.beg;
+  w.nq = (w.len + 127) >> 7;
+  w.head = local / w.nq;
+  w.k0 = (local - w.head * w.nq) * 128;
+  w.id = item;
+  return w;
+}
+
+__device__ __forceinline__ void bwd_store_item(volatile int32_t* d, const BwdItem& w) {
+  d[0] = w.seg; d[1] = w.beg; d[2] = w.len; d[3] = w.head; d[4] = w.k0; d[5] = w.nq; d[7] = w.id;
+}
+__device__ __forceinline__ BwdItem bwd_load_item(const volatile int32_t* d) {
+  BwdItem w;
+  w.seg = d[0]; w.beg = d[1]; w.len = d[2]; w.head = d[3]; w.k0 = d[4]; w.nq = d[5]; w.id = d[7];
+  return w;
+}
+
+// Next decoded item from the producer's ring: 1 with `w`, 0 when done, -2 when the wait gave up.
+__device__ __forceinline__ int bwd_next_item(BwdBars* bars, uint32_t& sk, const WaitCtl& wc, BwdItem& w) {
+  const int ss = sk & 1;
+  const uint32_t sph = (sk >> 1) & 1u;
+  ++sk;
+  if (!mbar_wait(&bars->sched_full[ss], sph, wc)) return -2;
+  w = bwd_load_item(bars->sched_item[ss]);
+  return w.seg < 0 ? 0 : 1;
+}
+
+__device__ __forceinline__ bool bwd_drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ producer
+template <int D>
+__device__ __forceinline__ void bwd_producer(const BwdParams& p, uint8_t* smem, BwdBars* bars, const WaitCtl& wc,
+                                             int32_t n_items, int32_t n_sorted) {
+  using C = BwdCfg<D>;
+  uint32_t sk = 0, kv_round = 0;
+  int qslot = 0;
+  uint32_t qphase = 0;
+  bool kv_armed = false;
+  uint32_t kv_armed_ph = 0, q_armed = 0, q_armed_ph = 0;
+  bool ok = true;
+  for (;;) {
+    const int ss = sk & 1;
+    const uint32_t sph = (sk >> 1) & 1u;
+    ++sk;
+    if (!(ok = mbar_wait(&bars->sched_empty[ss], sph ^ 1u, wc))) break;
+    const int32_t item = atomicAdd(p.next_item, 1);
+    BwdItem w;
+    if (item < n_items) {
+      w = bwd_decode_item(item, p, n_sorted);
+    } else {
+      w.seg = -1;
+    }
+    bwd_store_item(bars->sched_item[ss], w);
+    mbar_arrive(&bars->sched_full[ss]);
+    if (w.seg < 0) break;
+
+    const int32_t xcol = w.head * D;
+    if (!(ok = mbar_wait(&bars->kv_empty, (kv_round & 1u) ^ 1u, wc))) break;
+    mbar_arrive_expect_tx(&bars->kv_full, 2u * C::kTileBytes);
+    kv_armed = true;
+    kv_armed_ph = kv_round & 1u;
+    ++kv_round;
+#pragma unroll
+    for (int cb = 0; cb < C::kColBlocks; ++cb) {
+      tma_load_2d(smem + C::kOffK + cb * C::kBlockBytes, &p.tm_k, xcol + cb * 64, w.beg + w.k0, &bars->kv_full);
+      tma_load_2d(smem + C::kOffV + cb * C::kBlockBytes, &p.tm_v, xcol + cb * 64, w.beg + w.k0, &bars->kv_full);
+    }
+    for (int32_t i = 0; ok && i < w.nq; ++i) {
+      if (!(ok = mbar_wait(&bars->qd_empty[qslot], qphase ^ 1u, wc))) break;
+      mbar_arrive_expect_tx(&bars->qd_full[qslot], 2u * C::kTileBytes);
+      q_armed |= 1u << qslot;
+      q_armed_ph = (q_armed_ph & ~(1u << qslot)) | (qphase << qslot);
+#pragma unroll
+      for (int cb = 0; cb < C::kColBlocks; ++cb) {
+        tma_load_2d(smem + C::kOffQ + qslot * C::kTileBytes + cb * C::kBlockBytes, &p.tm_q, xcol + cb * 64,
+                    w.beg + i * 128, &bars->qd_full[qslot]);
+        tma_load_2d(smem + C::kOffDO + qslot * C::kTileBytes + cb * C::kBlockBytes, &p.tm_do, xcol + cb * 64,
+                    w.beg + i * 128, &bars->qd_full[qslot]);
+      }
+      if (++qslot == 2) {
+        qslot = 0;
+        qphase ^= 1u;
+      }
+    }
+    if (!ok) break;
+  }
+  if (!ok) {
+    // Let every copy this thread started land before the CTA can exit.
+    const uint64_t lim = wc.limit_ns;
+    if (kv_armed) bwd_drain_wait(&bars->kv_full, kv_armed_ph, lim);
+    for (int s = 0; s < 2; ++s)
+      if (q_armed & (1u << s)) bwd_drain_wait(&bars->qd_full[s], (q_armed_ph >> s) & 1u, lim);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+// A (M x K) from shared memory K-major, B (N x K) K-major: a score-like product
+// over d (S^T = K Q^T, dP^T = V dO^T).  N = 128.
+template <int D>
+__device__ __forceinline__ void bwd_issue_kmajor(uint32_t issue, uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+  constexpr uint32_t hi = sdesc_sw128_hi(1024);
+  const uint32_t a0 = sdesc_sw128_lo(a_addr, 16), b0 = sdesc_sw128_lo(b_addr, 16);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * BwdCfg<D>::kBlockBytes + (kk & 3) * 32) >> 4;
+    mma_bf16_ss_lo_if(issue, d_tmem, a0 + off, b0 + off, hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// D (+)= A B with A (128 rows x 128 along K) bf16 in tensor memory and B (K = 128
+// token rows x N = d) MN-major in shared memory: dV += P^T dO, dK += dS^T Q.
+template <int D>
+__device__ __forceinline__ void bwd_issue_tmem_a(uint32_t issue, uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr,
+                                                 bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
+  constexpr uint32_t hi = sdesc_sw128_hi(1024);
+  const uint32_t b0 = sdesc_sw128_lo(b_addr, BwdCfg<D>::kBlockBytes);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts_lo_if(issue, d_tmem, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
+                      (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// dQ = dS K: A = dS (M = 128 queries x K = 128 keys) read MN-major from the dS^T
+// buffer (rows = keys, queries contiguous), B = K (K = 128 keys x N = d) MN-major.
+template <int D>
+__device__ __forceinline__ void bwd_issue_dq(uint32_t issue, uint32_t d_tmem, uint32_t ds_addr, uint32_t k_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32_ab(128, D, true, true);
+  constexpr uint32_t hi = sdesc_sw128_hi(1024);
+  const uint32_t a0 = sdesc_sw128_lo(ds_addr, BwdCfg<D>::kBlockBytes);
+  const uint32_t b0 = sdesc_sw128_lo(k_addr, BwdCfg<D>::kBlockBytes);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk * 16 * 128) >> 4;
+    mma_bf16_ss_lo_if(issue, d_tmem, a0 + off, b0 + off, hi, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBars* bars, const WaitCtl& wc,
+                                        uint32_t tmem) {
+  using C = BwdCfg<D>;
+  const uint32_t k_addr = smem_u32(smem + C::kOffK);
+  const uint32_t v_addr = smem_u32(smem + C::kOffV);
+  const uint32_t q_addr0 = smem_u32(smem + C::kOffQ);
+  const uint32_t do_addr0 = smem_u32(smem + C::kOffDO);
+  const uint32_t ds_addr = smem_u32(smem + C::kOffDS);
+  uint32_t sk = 0, kv_round = 0, qphase = 0, pds_ph = 0, dqe_ph = 0, dkve_ph = 0;
+  int qslot = 0;
+  bool dq_pending = false, dkv_pending = false, ok = true;
+  const uint32_t leader = elect_one_sync();
+  for (;;) {
+    BwdItem w;
+    const int got = bwd_next_item(bars, sk, wc, w);
+    if (got != -2 && leader) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
+    if (got == -2) ok = false;
+    if (got <= 0) break;
+    if (!(ok = mbar_wait(&bars->kv_full, kv_round & 1u, wc))) break;
+    ++kv_round;
+    if (!(ok = mbar_wait(&bars->qd_full[qslot], qphase, wc))) break;
+    tc_fence_after();
+    bwd_issue_kmajor<D>(leader, tmem + C::kColA, k_addr, q_addr0 + qslot * C::kTileBytes);
+    for (int32_t i = 0; i < w.nq; ++i) {
+      const int cur = qslot;
+      if (dq_pending) {  // tensor memory B: the previous dQ partial has been read
+        if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
+        dqe_ph ^= 1u;
+        tc_fence_after();
+      }
+      bwd_issue_kmajor<D>(leader, tmem + C::kColB, v_addr, do_addr0 + cur * C::kTileBytes);
+      mma_commit_if(leader, &bars->s_full);
+      if (!(ok = mbar_wait(&bars->pds_full, pds_ph, wc))) break;
+      pds_ph ^= 1u;
+      tc_fence_after();
+      if (i == 0 && dkv_pending) {  // the previous item's dK, dV have been read
+        if (!(ok = mbar_wait(&bars->dkv_empty, dkve_ph, wc))) break;
+        dkve_ph ^= 1u;
+        tc_fence_after();
+      }
+      bwd_issue_tmem_a<D>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
+      bwd_issue_tmem_a<D>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
+      if (++qslot == 2) {
+        qslot = 0;
+        qphase ^= 1u;
+      }
+      if (i + 1 < w.nq) {
+        if (!(ok = mbar_wait(&bars->qd_full[qslot], qphase, wc))) break;
+        tc_fence_after();
+        bwd_issue_kmajor<D>(leader, tmem + C::kColA, k_addr, q_addr0 + qslot * C::kTileBytes);
+      }
+      bwd_issue_dq<D>(leader, tmem + C::kColB, ds_addr, k_addr);
+      mma_commit_if(leader, &bars->dq_full);
+      dq_pending = true;
+      mma_commit_if(leader, &bars->qd_empty[cur]);
+    }
+    if (!ok) break;
+    mma_commit_if(leader, &bars->dkv_full);
+    dkv_pending = true;
+    mma_commit_if(leader, &bars->kv_empty);
+  }
+  // Every MMA issued so far completes before tensor memory is released.
+  mma_commit_if(leader, &bars->drain);
+  bwd_drain_wait(&bars->drain, 0, wc.limit_ns);
+}
+
+// ------------------------------------------------------------------ elementwise: P^T, dS^T
+template <int D>
+__device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* smem, BwdBars* bars, const WaitCtl& wc,
+                                                uint32_t tmem) {
+  using C = BwdCfg<D>;
+  const int t = threadIdx.x & 127;  // key row of the tile (tensor-memory lane)
+  const int lane = threadIdx.x & 31;
+  const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
+  const uint32_t tA = tmem + lane_base + C::kColA;
+  const uint32_t tB = tmem + lane_base + C::kColB;
+  float* stage = reinterpret_cast<float*>(smem + C::kOffStage);  // [0,128): -lse2, [128,256): -D*scale
+  uint8_t* ds_row = smem + C::kOffDS + t * 128;
+  const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+  const uint64_t sc2 = f2_pack(p.scale, p.scale);
+  const uint64_t zero2 = 0;
+  uint32_t sk = 0, s_ph = 0, st_ph = 0;
+  for (;;) {
+    BwdItem w;
+    int got = bwd_next_item(bars, sk, wc, w);
+    if (__any_sync(0xffffffffu, got == -2)) got = -2;
+    __syncwarp();
+    if (lane == 0 && got != -2) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
+    if (got <= 0) break;
+    const bool key_ok = t < w.len - w.k0;
+    bool ok = true;
+    for (int32_t i = 0; i < w.nq; ++i) {
+      // the 128 queries' -lse2 and -D*scale (+inf lse past the segment end: P = 0)
+      const int32_t qrow = i * 128 + t;
+      float nl = -INFINITY, nd = 0.f;
+      if (qrow < w.len) {
+        const size_t hi = static_cast<size_t>(w.head) * p.total + w.beg + qrow;
+        nl = -__ldg(p.lse2 + hi);
+        nd = -__ldg(p.delta + hi) * p.scale;
+      }
+      // (bounded mbarrier waits, not named barriers: a warp that gives up must not
+      // leave the others blocked)
+      ok = mbar_wait(&bars->stage_empty, st_ph ^ 1u, wc);  // all warps are done with the last stage
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      stage[t] = nl;
+      stage[128 + t] = nd;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->stage_full);
+      ok = mbar_wait(&bars->stage_full, st_ph, wc);
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      st_ph ^= 1u;
+      ok = mbar_wait(&bars->s_full, s_ph, wc);
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      s_ph ^= 1u;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {  // 32 query columns per chunk
+        uint32_t sv[32], dpv[32];
+        PA_TMEM_LD32(tA + 32 * ch, sv);
+        PA_TMEM_LD32(tB + 32 * ch, dpv);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int q = 32 * ch + 2 * k;
+          const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(stage + q);
+          const uint64_t nd2 = *reinterpret_cast<const uint64_t*>(stage + 128 + q);
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
+          const uint64_t pp = ex2x2(x);
+          const uint64_t tt = f2_fma(f2_pack(__uint_as_float(dpv[2 * k]), __uint_as_float(dpv[2 * k + 1])), sc2, nd2);
+          const uint64_t ds = f2_fma(pp, tt, zero2);
+          pk[k] = key_ok ? pack_bf16x2_pair(pp) : 0u;
+          dk[k] = key_ok ? pack_bf16x2_pair(ds) : 0u;
+        }
+        PA_TMEM_ST16(tA + 16 * ch, pk);
+        PA_TMEM_ST16(tB + 16 * ch, dk);
+        // dS^T row t, queries 32ch .. 32ch+31, into the 128-byte-swizzled MN-major layout
+        uint8_t* blk = ds_row + (ch >> 1) * C::kBlockBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = (ch & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(blk + ((c ^ (t & 7)) << 4)) =
+              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->pds_full);
+        mbar_arrive(&bars->stage_empty);
+      }
+    }
+    if (!ok) break;
+  }
+}
+
+// ------------------------------------------------------------------ dQ reductions and dK, dV epilogue
+template <int D>
+__device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* bars, const WaitCtl& wc, uint32_t tmem) {
+  using C = BwdCfg<D>;
+  const int t = threadIdx.x & 127;
+  const int lane = threadIdx.x & 31;
+  const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
+  const uint32_t tB = tmem + lane_base + C::kColB;
+  const uint32_t tDV = tmem + lane_base + C::kColDV;
+  const uint32_t tDK = tmem + lane_base + C::kColDK;
+  uint32_t sk = 0, dqf_ph = 0, dkvf_ph = 0;
+  for (;;) {
+    BwdItem w;
+    int got = bwd_next_item(bars, sk, wc, w);
+    if (__any_sync(0xffffffffu, got == -2)) got = -2;
+    __syncwarp();
+    if (lane == 0 && got != -2) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
+    if (got <= 0) break;
+    bool ok = true;
+    for (int32_t i = 0; i < w.nq; ++i) {
+      ok = mbar_wait(&bars->dq_full, dqf_ph, wc);
+      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      dqf_ph ^= 1u;
+      tc_fence_after();
+      const int32_t qrow = i * 128 + t;
+      const bool row_ok = qrow < w.len;
+      const size_t tok = static_cast<size_t>(w.beg) + qrow;
+      float* base = p.dq_acc + (static_cast<size_t>(w.head) * (D / 4) * p.total + tok) * 4;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        PA_TMEM_LD32(tB + 32 * cc, o);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            red_add_v4_f32(base + static_cast<size_t>(cc * 8 + u) * p.total * 4, __uint_as_float(o[4 * u]),
+                           __uint_as_float(o[4 * u + 1]), __uint_as_float(o[4 * u + 2]),
+                           __uint_as_float(o[4 * u + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_empty);
+    }
+    if (!ok) break;
+    ok = mbar_wait(&bars->dkv_full, dkvf_ph, wc);
+    if (__any_sync(0xffffffffu, !ok)) break;
+    dkvf_ph ^= 1u;
+    tc_fence_after();
+    const bool key_ok = t < w.len - w.k0;
+    const size_t row = (static_cast<size_t>(w.beg + w.k0 + (key_ok ? t : 0)) * p.heads + w.head) * D;
+    uint4* dvp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dv) + row);
+    uint4* dkp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dk) + row);
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t a[32], b[32];
+      PA_TMEM_LD32(tDV + 32 * cc, a);
+      PA_TMEM_LD32(tDK + 32 * cc, b);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint4 va, vb;
+        va.x = pack_bf16x2(__uint_as_float(a[8 * u + 0]), __uint_as_float(a[8 * u + 1]));
+        va.y = pack_bf16x2(__uint_as_float(a[8 * u + 2]), __uint_as_float(a[8 * u + 3]));
+        va.z = pack_bf16x2(__uint_as_float(a[8 * u + 4]), __uint_as_float(a[8 * u + 5]));
+        va.w = pack_bf16x2(__uint_as_float(a[8 * u + 6]), __uint_as_float(a[8 * u + 7]));
+        vb.x = pack_bf16x2(__uint_as_float(b[8 * u + 0]), __uint_as_float(b[8 * u + 1]));
+        vb.y = pack_bf16x2(__uint_as_float(b[8 * u + 2]), __uint_as_float(b[8 * u + 3]));
+        vb.z = pack_bf16x2(__uint_as_float(b[8 * u + 4]), __uint_as_float(b[8 * u + 5]));
+        vb.w = pack_bf16x2(__uint_as_float(b[8 * u + 6]), __uint_as_float(b[8 * u + 7]));
+        if (key_ok) {
+          dvp[cc * 4 + u] = va;
+          dkp[cc * 4 + u] = vb;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->dkv_empty);
+  }
+}
+
+// ------------------------------------------------------------------ kernels
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::kOffBar);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qd_full[s], 1);
+      mbar_init(&bars->qd_empty[s], 1);
+      mbar_init(&bars->sched_full[s], 1);
+      mbar_init(&bars->sched_empty[s], 9);  // the MMA warp + one lane of each of 8 warps
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->pds_full, 4);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 4);
+    mbar_init(&bars->dkv_full, 1);
+    mbar_init(&bars->dkv_empty, 4);
+    mbar_init(&bars->stage_full, 4);
+    mbar_init(&bars->stage_empty, 4);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const WaitCtl wc{&bars->abort_flag, p.status, p.wait_limit_ns, p.err_timeout};
+  const int32_t n_items = p.counts[0];
+  const int32_t n_sorted = p.counts[1];
+  if (warp < 8) {
+    regs_increase<kBwdMathRegs>();
+    if (warp < 4) bwd_elementwise<D>(p, smem, bars, wc, tmem);
+    else bwd_reduce_store<D>(p, bars, wc, tmem);
+    tc_fence_before();
+    named_bar_sync(1, kBwdThreads);
+  } else {
+    regs_decrease<kBwdControlRegs>();
+    if (warp == 8) {
+      if ((threadIdx.x & 31) == 0) bwd_producer<D>(p, smem, bars, wc, n_items, n_sorted);
+    } else if (warp == 9) {
+      bwd_mma<D>(p, smem, bars, wc, tmem);  // the whole warp; one elected lane issues
+    }
+    __syncwarp();
+    tc_fence_before();
+    named_bar_sync(1, kBwdThreads);
+    if (warp == 9) {
+      tc_fence_after();
+      tmem_dealloc(tmem, C::kTmemCols);
+    }
+  }
+}
+
+// D = dout . out per (token, head) and lse * log2(e), both written head-major [H][T].
+// One warp per (token, head) row.
+template <int D>
+__global__ void bwd_prep_kernel(const uint16_t* __restrict__ out, const uint16_t* __restrict__ dout,
+                                const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
+                                int32_t total, int32_t heads) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<int64_t>(total) * heads) return;
+  const int32_t tok = static_cast<int32_t>(row / heads), h = static_cast<int32_t>(row - static_cast<int64_t>(tok) * heads);
+  constexpr int kPer = D / 32;  // bf16 elements per lane
+  const uint16_t* o = out + row * D + lane * kPer;
+  const uint16_t* g = dout + row * D + lane * kPer;
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e)
+    acc += __uint_as_float(static_cast<uint32_t>(o[e]) << 16) * __uint_as_float(static_cast<uint32_t>(g[e]) << 16);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) {
+    const size_t hi = static_cast<size_t>(h) * total + tok;
+    delta[hi] = acc;
+    lse2[hi] = lse[row] * 1.4426950408889634f;
+  }
+}
+
+// dq [T, H, d] bf16 from the fp32 accumulator [H][d/4][T] x 4; one thread per float4.
+template <int D>
+__global__ void bwd_dq_convert_kernel(const float4* __restrict__ acc, uint16_t* __restrict__ dq, int32_t total,
+                                      int32_t heads) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(total) * heads * (D / 4);
+  if (idx >= n) return;
+  const int32_t tok = static_cast<int32_t>(idx % total);
+  const int64_t hc = idx / total;  // h * (D/4) + c4
+  const int32_t h = static_cast<int32_t>(hc / (D / 4)), c4 = static_cast<int32_t>(hc % (D / 4));
+  const float4 v = acc[idx];
+  uint2 pk;
+  pk.x = pack_bf16x2(v.x, v.y);
+  pk.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(dq + (static_cast<size_t>(tok) * heads + h) * D + c4 * 4) = pk;
+}
+
+}  // namespace pa

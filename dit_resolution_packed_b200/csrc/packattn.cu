@@ -15,6 +15,7 @@
 #include <mutex>
 #include <vector>
 
+#include "attn_bwd_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "packattn.h"
 #include "schedule.cuh"
@@ -128,6 +129,12 @@ int ensure_device(int device) {
   if (cudaFuncSetAttribute(pa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            pa::FwdCfg<128>::kSmemBytes) != cudaSuccess)
     return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::BwdCfg<64>::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::BwdCfg<128>::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
   d.ready = true;
   return PA_OK;
 }
@@ -145,6 +152,25 @@ bool encode_map(CUtensorMap* m, const void* base, int32_t rows, int32_t heads, i
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Backward workspace: the schedule, then lse * log2(e) and D head-major [H][T],
+// then the fp32 dq accumulator [H][d/4][T] x 4.
+struct BwdWsLayout {
+  size_t counts, order, item_start, lse2, delta, dq_acc, total;
+};
+
+BwdWsLayout bwd_ws_layout(int32_t batch, int32_t total, int32_t heads, int32_t head_dim) {
+  BwdWsLayout L;
+  const size_t rows = static_cast<size_t>(total) * heads;
+  L.counts = 0;
+  L.order = 128;
+  L.item_start = align_up(L.order + 4 * static_cast<size_t>(batch), 128);
+  L.lse2 = align_up(L.item_start + 4 * (static_cast<size_t>(batch) + 1), 256);
+  L.delta = align_up(L.lse2 + 4 * rows, 256);
+  L.dq_acc = align_up(L.delta + 4 * rows, 256);
+  L.total = L.dq_acc + 4 * rows * static_cast<size_t>(head_dim);
+  return L;
+}
 
 }  // namespace
 
@@ -237,6 +263,7 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
   sp.total = total_tokens;
   sp.heads = heads;
   sp.max_seqlen = max_seqlen;
+  sp.rows_log2 = 8;
   sp.err_cu = PA_ERR_CU_SEQLENS;
   sp.err_max = PA_ERR_MAX_SEQLEN;
   pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
@@ -287,6 +314,121 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
   if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (g_prof_on) cudaEventRecord(ev1, stream);
   return PA_OK;
+}
+
+int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                       const void* dout, const int32_t* cu_seqlens, int32_t batch, int32_t total_tokens,
+                       int32_t heads, int32_t head_dim, int32_t max_seqlen, float scale, void* dq, void* dk,
+                       void* dv, void* stream_handle) {
+  // ---- host-visible argument checks: nothing is enqueued on failure
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SCALE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  if (max_seqlen < 1) return PA_ERR_MAX_SEQLEN;
+  if (!q || !k || !v || !out || !lse || !dout || !cu_seqlens || !dq || !dk || !dv) return PA_ERR_NULL;
+  const void* a16[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* ptr : a16)
+    if (!aligned(ptr, 16)) return PA_ERR_ALIGN;
+  if (!aligned(lse, 4) || !aligned(cu_seqlens, 4)) return PA_ERR_ALIGN;
+  const int64_t item_bound = static_cast<int64_t>(heads) * ((static_cast<int64_t>(total_tokens) + 127) / 128 + batch);
+  if (item_bound >= (int64_t(1) << 31) || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24) ||
+      static_cast<int64_t>(total_tokens) * heads * head_dim >= (int64_t(1) << 40))
+    return PA_ERR_SHAPE;
+
+  int dev = -1, d2 = -1;
+  int rc;
+  if ((rc = device_of(q, &dev)) != PA_OK) return rc;
+  const void* others[10] = {k, v, out, lse, dout, cu_seqlens, dq, dk, dv, q};
+  for (const void* ptr : others) {
+    if ((rc = device_of(ptr, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  const BwdWsLayout L = bwd_ws_layout(batch, total_tokens, heads, head_dim);
+  if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
+
+  pa::BwdParams bp;
+  std::memset(&bp, 0, sizeof(bp));
+  if (!encode_map(&bp.tm_q, q, total_tokens, heads, head_dim) || !encode_map(&bp.tm_k, k, total_tokens, heads, head_dim) ||
+      !encode_map(&bp.tm_v, v, total_tokens, heads, head_dim) ||
+      !encode_map(&bp.tm_do, dout, total_tokens, heads, head_dim))
+    return PA_ERR_CUDA;
+  float* lse2 = reinterpret_cast<float*>(st->ws + L.lse2);
+  float* delta = reinterpret_cast<float*>(st->ws + L.delta);
+  float* dq_acc = reinterpret_cast<float*>(st->ws + L.dq_acc);
+  const size_t rows = static_cast<size_t>(total_tokens) * heads;
+
+  if (cudaMemsetAsync(dq_acc, 0, 4 * rows * static_cast<size_t>(head_dim), stream) != cudaSuccess) return PA_ERR_CUDA;
+  const unsigned prep_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (head_dim == 128)
+    pa::bwd_prep_kernel<128><<<prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
+                                                            static_cast<const uint16_t*>(dout), lse, delta, lse2,
+                                                            total_tokens, heads);
+  else
+    pa::bwd_prep_kernel<64><<<prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
+                                                           static_cast<const uint16_t*>(dout), lse, delta, lse2,
+                                                           total_tokens, heads);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  pa::SchedParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  sp.cu = cu_seqlens;
+  sp.status = st->status;
+  sp.counts = reinterpret_cast<int32_t*>(st->ws + L.counts);
+  sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
+  sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
+  sp.maps = nullptr;
+  sp.batch = batch;
+  sp.total = total_tokens;
+  sp.heads = heads;
+  sp.max_seqlen = max_seqlen;
+  sp.rows_log2 = 7;
+  sp.err_cu = PA_ERR_CU_SEQLENS;
+  sp.err_max = PA_ERR_MAX_SEQLEN;
+  pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  bp.cu = cu_seqlens;
+  bp.counts = sp.counts;
+  bp.next_item = sp.counts + 2;
+  bp.order = sp.order;
+  bp.item_start = sp.item_start;
+  bp.lse2 = lse2;
+  bp.delta = delta;
+  bp.dq_acc = dq_acc;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.status = st->status;
+  bp.heads = heads;
+  bp.total = total_tokens;
+  bp.scale = scale;
+  bp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  bp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  bp.err_timeout = PA_ERR_TIMEOUT;
+  const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
+  if (head_dim == 128)
+    pa::attn_bwd_kernel<128><<<grid, pa::kBwdThreads, pa::BwdCfg<128>::kSmemBytes, stream>>>(bp);
+  else
+    pa::attn_bwd_kernel<64><<<grid, pa::kBwdThreads, pa::BwdCfg<64>::kSmemBytes, stream>>>(bp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  const size_t n4 = rows * static_cast<size_t>(head_dim / 4);
+  const unsigned conv_blocks = static_cast<unsigned>((n4 + 255) / 256);
+  if (head_dim == 128)
+    pa::bwd_dq_convert_kernel<128><<<conv_blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                                  static_cast<uint16_t*>(dq), total_tokens, heads);
+  else
+    pa::bwd_dq_convert_kernel<64><<<conv_blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                                 static_cast<uint16_t*>(dq), total_tokens, heads);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int pa_get_error(void* stream_handle) {
@@ -447,6 +589,7 @@ int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, cons
   sp.total = total_tokens;
   sp.heads = heads;
   sp.max_seqlen = max_seqlen;
+  sp.rows_log2 = 8;
   sp.err_cu = PA_ERR_CU_SEQLENS;
   sp.err_max = PA_ERR_MAX_SEQLEN;
   pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);

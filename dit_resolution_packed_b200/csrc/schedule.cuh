@@ -9,12 +9,13 @@
 //      number of 128-key tiles, i.e. on the per-item cost), so a persistent grid
 //      takes the big items first (longest-processing-time order);
 //   3. publishes, in that order, the first work-item index of every segment;
-//      a segment of L tokens holds heads * ceil(L / 256) items, one per
-//      (head, pair of 128-row query tiles);
-//   4. writes three tensor maps per segment (q, k, v) whose base is the
-//      segment's first token and whose row extent is L, so that every TMA tile
-//      stops at the segment boundary: loads past it read zeros and no tile
-//      touches another image.
+//      a segment of L tokens holds heads * ceil(L / 2^rows_log2) items: for the
+//      forward (rows_log2 = 8) one per (head, pair of 128-row query tiles), for
+//      the backward (rows_log2 = 7) one per (head, 128-key tile);
+//   4. for the forward, writes three tensor maps per segment (q, k, v) whose
+//      base is the segment's first token and whose row extent is L, so that
+//      every TMA tile stops at the segment boundary: loads past it read zeros
+//      and no tile touches another image (maps == nullptr skips this step).
 //
 // The mask of the method (Mage-Flow page, "Packing + Flash Attention varlen":
 // images attend only to themselves, no padding) is thereby carried entirely by
@@ -40,9 +41,10 @@ struct SchedParams {
   int32_t* counts;         // [0] = work items, [1] = non-empty segments, [2] = work counter (zeroed)
   int32_t* order;          // [B] segment ids, longest first
   int32_t* item_start;     // [B+1] first item of each ordered segment
-  uint8_t* maps;           // [B][3] tensor maps, 128 bytes each
+  uint8_t* maps;           // [B][3] tensor maps, 128 bytes each (nullptr: none)
   uint64_t row_bytes;      // H * d * 2
   int32_t batch, total, heads, max_seqlen;
+  int32_t rows_log2;        // rows of a work item: 2^rows_log2 (8 forward, 7 backward)
   int32_t err_cu, err_max;  // status codes to record
 };
 
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   }
 
   // 2. per-segment tensor maps: copy the template, then move its base and row extent
-  for (int idx = tid; idx < 3 * B; idx += kSchedThreads) {
+  for (int idx = tid; p.maps != nullptr && idx < 3 * B; idx += kSchedThreads) {
     const int s = idx / 3, which = idx - 3 * s;
     const int32_t beg = cu[s], len = cu[s + 1] - beg;
     if (len <= 0) continue;
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     if (k < n_sorted) {
       const int s = p.order[k];
       const int32_t len = cu[s + 1] - cu[s];
-      items = static_cast<int64_t>(p.heads) * ((len + 255) >> 8);
+      items = static_cast<int64_t>(p.heads) * ((static_cast<int64_t>(len) + (1 << p.rows_log2) - 1) >> p.rows_log2);
     }
     const int64_t ex = block_exclusive_scan(items, s_warp, &s_total);
     if (k < n_sorted) p.item_start[k] = static_cast<int32_t>(carry + ex);

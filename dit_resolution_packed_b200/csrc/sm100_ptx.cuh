@@ -272,6 +272,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) |
          ((M >> 4) << 24);
 }
+// The same with the major-ness of A chosen too (bit 15: 1 = A is MN-major in shared memory).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(uint32_t M, uint32_t N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand:
 //   bits 0-13 start address >> 4; 16-29 leading byte offset >> 4; 32-45 stride
@@ -409,6 +413,12 @@ __device__ __forceinline__ void tmem_ld128_pairs(uint32_t taddr, uint64_t (&v)[6
       : "=l"(v[0]), "=l"(v[1]), "=l"(v[2]), "=l"(v[3]), "=l"(v[4]), "=l"(v[5]), "=l"(v[6]), "=l"(v[7]), "=l"(v[8]), "=l"(v[9]), "=l"(v[10]), "=l"(v[11]), "=l"(v[12]), "=l"(v[13]), "=l"(v[14]), "=l"(v[15]), "=l"(v[16]), "=l"(v[17]), "=l"(v[18]), "=l"(v[19]), "=l"(v[20]), "=l"(v[21]), "=l"(v[22]), "=l"(v[23]), "=l"(v[24]), "=l"(v[25]), "=l"(v[26]), "=l"(v[27]), "=l"(v[28]), "=l"(v[29]), "=l"(v[30]), "=l"(v[31]), "=l"(v[32]), "=l"(v[33]), "=l"(v[34]), "=l"(v[35]), "=l"(v[36]), "=l"(v[37]), "=l"(v[38]), "=l"(v[39]), "=l"(v[40]), "=l"(v[41]), "=l"(v[42]), "=l"(v[43]), "=l"(v[44]), "=l"(v[45]), "=l"(v[46]), "=l"(v[47]), "=l"(v[48]), "=l"(v[49]), "=l"(v[50]), "=l"(v[51]), "=l"(v[52]), "=l"(v[53]), "=l"(v[54]), "=l"(v[55]), "=l"(v[56]), "=l"(v[57]), "=l"(v[58]), "=l"(v[59]), "=l"(v[60]), "=l"(v[61]), "=l"(v[62]), "=l"(v[63])
       : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
       : "memory");
+}
+
+// *addr += {a, b, c, d} (four fp32 reductions in one request, in L2; relaxed).
+__device__ __forceinline__ void red_add_v4_f32(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

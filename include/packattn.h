@@ -86,6 +86,38 @@ PA_API int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const
                               int32_t max_seqlen, float scale, void* out, float* lse, void* stream);
 
 /*
+ * pa_varlen_attn_bwd -- enqueue the gradients of pa_varlen_attn_fwd on `stream`:
+ * dq, dk, dv from q, k, v, the forward's out and lse, and dout = dL/dout.
+ * (Chain rule through the row softmax of the forward definition, SparseAttn page,
+ * section 3.1; P recomputed from the saved log-sum-exp as in the blockwise
+ * algorithm of the GigaPath-Flash page, sections 3.2 / 4.2.)  Per segment, head,
+ * query row r and key j of the segment:
+ *     P_rj  = exp(scale * q_r . k_j - lse_r),     D_r = dout_r . out_r,
+ *     dS_rj = P_rj (dout_r . v_j - D_r),
+ *     dq_r  = scale * sum_j dS_rj k_j,   dk_j = scale * sum_r dS_rj q_r,
+ *     dv_j  = sum_r P_rj dout_r.
+ *
+ *   q, k, v, out, dout   device, bf16, [total_tokens, heads, head_dim], contiguous,
+ *                        16-byte aligned; out and lse as pa_varlen_attn_fwd wrote
+ *                        them for the same q, k, v, cu_seqlens and scale.
+ *   lse                  device, fp32, [total_tokens, heads], 4-byte aligned.
+ *   cu_seqlens, batch, total_tokens, heads, head_dim, max_seqlen, scale:
+ *                        as for pa_varlen_attn_fwd.
+ *   dq, dk, dv           device, bf16, [total_tokens, heads, head_dim], 16-byte
+ *                        aligned, written (each rounded once to nearest even).
+ *
+ * Ownership, workspace and errors: as for pa_varlen_attn_fwd.  The workspace of
+ * the (device, stream) pair also holds an fp32 dq accumulator of
+ * 4 * total_tokens * heads * head_dim bytes.  dk and dv are bitwise
+ * deterministic; dq sums fp32 partials of different key tiles in whatever order
+ * they arrive, so its last bits may differ from run to run.
+ */
+PA_API int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                              const void* dout, const int32_t* cu_seqlens, int32_t batch, int32_t total_tokens,
+                              int32_t heads, int32_t head_dim, int32_t max_seqlen, float scale, void* dq, void* dk,
+                              void* dv, void* stream);
+
+/*
  * pa_get_error -- synchronise `stream`, return the first device-side error
  * recorded for the calling device and `stream` since the last call (PA_OK if
  * none) and clear it.  Returns PA_ERR_CUDA if the synchronisation fails.

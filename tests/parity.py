@@ -53,3 +53,35 @@ def gather_rows(out, lse, tok, head):
     t = torch.as_tensor(tok, dtype=torch.long, device=out.device)
     h = torch.as_tensor(head, dtype=torch.long, device=out.device)
     return (out[t, h].double().cpu().numpy(), lse[t, h].double().cpu().numpy())
+
+
+# ---- gradients (pa_varlen_attn_bwd) against the fp64 gradient oracle
+#
+# No tolerance is given for the gradients; this one follows from the arithmetic.
+# With u = 2^-9 (bf16 unit roundoff): P and dS are rounded to bf16 before the
+# MMAs (one rounding per product term, u relative), D = dout . out uses the
+# forward's bf16-rounded out (u relative in each term), the partial sums run in
+# fp32, and each gradient is rounded to bf16 once (u).  The rounding errors of
+# the terms are independent, so in the Frobenius norm they add to a few u:
+# relative Frobenius error <= 1e-2 (about 5u).  Element-wise, a gradient can be
+# a small difference of larger terms, so the bound is taken relative to the
+# tensor's largest magnitude: |err| <= 2e-2 * max|ref| (about 10u).
+BWD_REL_FRO = 1e-2
+BWD_MAX_REL = 2e-2
+
+
+def bwd_errors(got, ref):
+    g = np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    d = g - r
+    scale = float(np.max(np.abs(r))) if r.size else 0.0
+    den = float(np.linalg.norm(r))
+    return dict(max_abs=float(np.max(np.abs(d))) if d.size else 0.0, ref_max=scale,
+                rel_fro=float(np.linalg.norm(d) / den) if den > 0 else float(np.linalg.norm(d)),
+                finite=bool(np.all(np.isfinite(g))))
+
+
+def bwd_check(errs, name=""):
+    assert errs["finite"], (name, errs)
+    assert errs["rel_fro"] <= BWD_REL_FRO, (name, errs)
+    assert errs["max_abs"] <= BWD_MAX_REL * errs["ref_max"] + 1e-30, (name, errs)

@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 10
+    assert len(names) == len(set(names)) == 11
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -75,6 +75,24 @@ def test_noalloc_rejects_batch_above_its_limit_before_any_cuda_call(lib):
     assert f(*args(1 << 30)) == pa.PA_ERR_NOALLOC_LIMIT
     assert f(*args(pa.NOALLOC_MAX_BATCH, head_dim=96)) == pa.PA_ERR_HEAD_DIM
     assert f(16, 16, 16, 16, 3, 0, 1, 64, 4, ctypes.c_float(0.125), 16, 16, None, None) == pa.PA_OK
+
+
+def test_bwd_host_validation_before_any_cuda_call(lib):
+    def raw(q=16, out=16, lse=16, dout=16, batch=1, total=4, heads=1, head_dim=64, max_seqlen=4, scale=0.125,
+            dq=16):
+        return lib.pa_varlen_attn_bwd(q, 16, 16, out, lse, dout, 16, batch, total, heads, head_dim, max_seqlen,
+                                      ctypes.c_float(scale), dq, 16, 16, None)
+    assert raw(head_dim=80) == pa.PA_ERR_HEAD_DIM
+    assert raw(heads=0) == pa.PA_ERR_SHAPE
+    assert raw(batch=0, total=3) == pa.PA_ERR_SHAPE
+    assert raw(batch=0, total=0) == pa.PA_OK
+    assert raw(scale=math.inf) == pa.PA_ERR_SCALE
+    assert raw(max_seqlen=0) == pa.PA_ERR_MAX_SEQLEN
+    assert raw(dout=None) == pa.PA_ERR_NULL
+    assert raw(lse=None) == pa.PA_ERR_NULL
+    assert raw(dq=24) == pa.PA_ERR_ALIGN
+    assert raw(out=8) == pa.PA_ERR_ALIGN
+    assert raw(lse=18) == pa.PA_ERR_ALIGN
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -104,6 +104,13 @@ def sampled_rows(cfg, per_head=None):
     return torch.cat(toks), torch.cat(heads)
 
 
+def random_dout(shape, seed):
+    """The upstream gradient dL/dout of a backward workload: N(0,1) in fp32 from its own
+    seeded CPU generator, rounded to bf16."""
+    g = torch.Generator().manual_seed(int(seed))
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
 def random_pack(lengths, heads, head_dim, seed, scale=None):
     """An ad-hoc pack of the given segment lengths with seeded N(0,1) bf16 inputs."""
     lengths = [int(n) for n in lengths]
