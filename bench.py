@@ -295,6 +295,48 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
     value = flops * world / (ms_per_step * 1e-3) / 1e12
 
+    # ---- backward (the gradients of the same call): out and lse from the forward above, dout a
+    # seeded N(0,1) tensor; same warm-up, step count and L2 flush as the forward
+    dout = workloads.random_dout(q.shape, 7919 + rank).to(device)
+    gq, gk, gv = (torch.empty_like(q) for _ in range(3))
+
+    def bwd_call():
+        rc = pa.pa_varlen_attn_bwd(q, k, v, out, lse, dout, cu, p["max_seqlen"], p["scale"], gq, gk, gv, stream)
+        if rc != pa.PA_OK:
+            raise pa.PackAttnError(rc, "pa_varlen_attn_bwd")
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        bwd_call()
+    torch.cuda.synchronize()
+    bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(1.0)
+        bev[i][0].record(stream)
+        bwd_call()
+        bev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    bwd_step_ms = [a.elapsed_time(b) for a, b in bev]
+    pa.pa_profile_read()  # clear
+    pa.pa_profile_enable(True)
+    t_bprof0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(1.0)
+        bwd_call()
+    torch.cuda.synchronize()
+    t_bprof = time.time() - t_bprof0
+    pa.pa_profile_enable(False)
+    bkern_ms_total, bkern_n = pa.pa_profile_read()
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, "backward region")
+    bwd_flops = 2.5 * flops  # five GEMMs (S^T, dP^T, dV, dK, dQ) against the forward's two
+    bwd_ms = allreduce_max(sum(bwd_step_ms), world, device) / args.steps
+    bq10, bq50, bq90 = (float(x) for x in np.percentile(bwd_step_ms, [10, 50, 90]))
+
     # ---- end to end through the public API with host buffers (pinned): every step copies its
     # q, k, v, cu_seqlens host -> device and its out, lse device -> host inside the timed region.
     # Steps are pipelined the way an input pipeline runs them: two device buffer sets and three
@@ -362,6 +404,10 @@ def run_ours(args, world, rank, local):
     # long enough to settle under the board's power limit (>= 0.25 s), its denominator is
     # the sustained cuBLAS figure, else the burst one.
     sustained = t_prof >= 0.25
+    bpeak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])) \
+        if t_bprof >= 0.25 else peak_burst
+    bpeak_src = (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_bprof:.2f} s of back-to-back steps)"
+                 if t_bprof >= 0.25 else f"bf16_tflops ({peak_src}, burst)")
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])) if sustained \
         else peak_burst
     trec = traffic_for_current_kernel()
@@ -390,6 +436,17 @@ def run_ours(args, world, rank, local):
                 "pipelining": "two device buffer sets, three streams: the copies of steps i-1 and i+1 "
                               "overlap the kernels of step i; one region timed over all steps",
                 "l2": "not flushed: each step's inputs arrive by host-to-device copy"},
+        "backward": {
+            "metric": "varlen attn bwd effective TFLOP/s (valid FLOPs: 5 GEMMs = 10 * sum(L_i^2) * d * H)",
+            "value": bwd_flops * world / (bwd_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": bwd_ms,
+            "step_ms_p10_p50_p90": [bq10, bq50, bq90], "valid_flops_per_step": bwd_flops,
+            "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel<%d>" % d,
+                         "achieved": bwd_flops / (bkern_ms_total / max(1, bkern_n) * 1e-3) / 1e12,
+                         "peak": bpeak, "unit": "TFLOP/s",
+                         "frac": bwd_flops / (bkern_ms_total / max(1, bkern_n) * 1e-3) / 1e12 / bpeak,
+                         "peak_source": bpeak_src, "traffic": None},
+            "gpu_launches": 4 * args.steps,  # prep, schedule, main, dq conversion per step
+        },
         "gpu_launches": 2 * args.steps,  # schedule + attention kernel per step, headline timed region
         "clocks": clock_rec,
     }

@@ -414,11 +414,23 @@ int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* 
   bp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
   bp.err_timeout = PA_ERR_TIMEOUT;
   const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
+  cudaEvent_t ev1 = nullptr;
+  if (g_prof_on) {  // events around the backward main kernel, as for the forward
+    if (g_prof_used == g_prof_events.size()) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return PA_ERR_CUDA;
+      g_prof_events.emplace_back(a, b);
+    }
+    cudaEventRecord(g_prof_events[g_prof_used].first, stream);
+    ev1 = g_prof_events[g_prof_used].second;
+    ++g_prof_used;
+  }
   if (head_dim == 128)
     pa::attn_bwd_kernel<128><<<grid, pa::kBwdThreads, pa::BwdCfg<128>::kSmemBytes, stream>>>(bp);
   else
     pa::attn_bwd_kernel<64><<<grid, pa::kBwdThreads, pa::BwdCfg<64>::kSmemBytes, stream>>>(bp);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (ev1) cudaEventRecord(ev1, stream);
 
   const size_t n4 = rows * static_cast<size_t>(head_dim / 4);
   const unsigned conv_blocks = static_cast<unsigned>((n4 + 255) / 256);

@@ -155,7 +155,9 @@ PA_API int pa_selftest_wait_timeout(uint32_t limit_us, void* stream);
  * Kernel timing for measurement.  While enabled, pa_varlen_attn_fwd records a
  * pair of CUDA events on its stream around the attention kernel (not the
  * schedule kernel) and launches it without overlapping the schedule kernel
- * (no programmatic dependent launch), so the events bracket it alone.  pa_profile_read synchronises on the last recorded event,
+ * (no programmatic dependent launch), so the events bracket it alone;
+ * pa_varlen_attn_bwd records a pair around its main kernel (not the prep,
+ * schedule and dq conversion kernels).  pa_profile_read synchronises on the last recorded event,
  * writes the summed attention-kernel time in milliseconds and the number of
  * launches timed, and clears the record.  Returns PA_OK or PA_ERR_CUDA.
  */
