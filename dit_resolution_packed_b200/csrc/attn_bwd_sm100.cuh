@@ -19,7 +19,7 @@
 //     dV  += P^T dO       (A = P^T bf16 in TMEM A, B = dO MN-major)
 //     dK  += dS^T Q       (A = dS^T bf16 in TMEM B, B = Q MN-major)
 //     dQ   = dS K         (A = dS^T in shared memory, read MN-major; B = K MN-major) -> TMEM B
-// and the next tile's S^T is issued between dK and dQ.  The dQ partial of every
+// and then the next tile's S^T (so the read-out of dQ overlaps it).  The dQ partial of every
 // (key tile, query tile) is added into an fp32 accumulator laid out [H][d/4][T]
 // (float4 per element group, token fastest), so that the 32 reductions of a warp
 // cover 512 contiguous bytes; a last kernel converts it to bf16 [T, H, d].
@@ -309,6 +309,11 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
       }
       bwd_issue_tmem_a<D>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
       bwd_issue_tmem_a<D>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
+      // dQ before the next S^T, so that its read-out overlaps that MMA
+      bwd_issue_dq<D>(leader, tmem + C::kColB, ds_addr, k_addr);
+      mma_commit_if(leader, &bars->dq_full);
+      dq_pending = true;
+      mma_commit_if(leader, &bars->qd_empty[cur]);
       if (++qslot == 2) {
         qslot = 0;
         qphase ^= 1u;
@@ -318,10 +323,6 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
         tc_fence_after();
         bwd_issue_kmajor<D>(leader, tmem + C::kColA, k_addr, q_addr0 + qslot * C::kTileBytes);
       }
-      bwd_issue_dq<D>(leader, tmem + C::kColB, ds_addr, k_addr);
-      mma_commit_if(leader, &bars->dq_full);
-      dq_pending = true;
-      mma_commit_if(leader, &bars->qd_empty[cur]);
     }
     if (!ok) break;
     mma_commit_if(leader, &bars->dkv_full);
@@ -382,12 +383,20 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       s_ph ^= 1u;
       tc_fence_after();
+      // 32 query columns per chunk; the loads of chunk ch + 1 are in flight while chunk ch
+      // is computed (they read columns 32(ch+1).., the stores of chunk ch write 16ch..16ch+15)
+      uint32_t sbuf[2][32], dbuf[2][32];
+      PA_TMEM_LD32(tA, sbuf[0]);
+      PA_TMEM_LD32(tB, dbuf[0]);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {  // 32 query columns per chunk
-        uint32_t sv[32], dpv[32];
-        PA_TMEM_LD32(tA + 32 * ch, sv);
-        PA_TMEM_LD32(tB + 32 * ch, dpv);
+      for (int ch = 0; ch < 4; ++ch) {
         tmem_wait_ld();
+        if (ch < 3) {
+          PA_TMEM_LD32(tA + 32 * (ch + 1), sbuf[(ch + 1) & 1]);
+          PA_TMEM_LD32(tB + 32 * (ch + 1), dbuf[(ch + 1) & 1]);
+        }
+        const uint32_t (&sv)[32] = sbuf[ch & 1];
+        const uint32_t (&dpv)[32] = dbuf[ch & 1];
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -453,22 +462,20 @@ __device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* ba
       const bool row_ok = qrow < w.len;
       const size_t tok = static_cast<size_t>(w.beg) + qrow;
       float* base = p.dq_acc + (static_cast<size_t>(w.head) * (D / 4) * p.total + tok) * 4;
+      uint32_t o[D];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        PA_TMEM_LD32(tB + 32 * cc, o);
-        tmem_wait_ld();
-        if (row_ok) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            red_add_v4_f32(base + static_cast<size_t>(cc * 8 + u) * p.total * 4, __uint_as_float(o[4 * u]),
-                           __uint_as_float(o[4 * u + 1]), __uint_as_float(o[4 * u + 2]),
-                           __uint_as_float(o[4 * u + 3]));
-        }
-      }
+      for (int cc = 0; cc < D / 32; ++cc) PA_TMEM_LD32(tB + 32 * cc, (o + 32 * cc));
+      tmem_wait_ld();
+      // the columns are free as soon as they are in registers
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_empty);
+      if (row_ok) {
+#pragma unroll
+        for (int u = 0; u < D / 4; ++u)
+          red_add_v4_f32(base + static_cast<size_t>(u) * p.total * 4, __uint_as_float(o[4 * u]),
+                         __uint_as_float(o[4 * u + 1]), __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
+      }
     }
     if (!ok) break;
     ok = mbar_wait(&bars->dkv_full, dkvf_ph, wc);
