@@ -459,6 +459,67 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_packing_study(args, local):
+    """Padded vs bucketed vs packed (Mage-Flow page, the table after "Packing + Flash Attention
+    varlen"): the training pack's images through the forward + backward of the packed kernel,
+    laid out three ways.  The padded and bucketed layouts run every padded sequence as a
+    segment of its padded length: the work of a dense kernel over padded sequences (their
+    outputs are a timing vehicle, not compared).  Prints one JSON line."""
+    import dit_resolution_packed_b200 as pa
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    cfg = workloads.load_config(args.config if args.config != "mixed" else "training")
+    H, d = cfg["heads"], cfg["head_dim"]
+    real = [int(n) for n in cfg["segments"]]
+    valid = workloads.valid_flops(real, H, d)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, lay in workloads.packing_layouts(real).items():
+        p = workloads.random_pack(lay["segments"], H, d, seed=int(cfg["seed"]), scale=cfg["scale"])
+        q, k, v = (p[n].to(device) for n in ("q", "k", "v"))
+        cu = p["cu_seqlens"].to(device)
+        out, lse = torch.empty_like(q), torch.empty(q.shape[0], H, dtype=torch.float32, device=device)
+        dout = workloads.random_dout(q.shape, 11).to(device)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+
+        def step():
+            rc = pa.pa_varlen_attn_fwd(q, k, v, cu, p["max_seqlen"], p["scale"], out, lse, stream)
+            rc = rc or pa.pa_varlen_attn_bwd(q, k, v, out, lse, dout, cu, p["max_seqlen"], p["scale"], dq, dk, dv,
+                                             stream)
+            if rc != pa.PA_OK:
+                raise pa.PackAttnError(rc, name)
+
+        n_steps = max(10, args.steps // 30)
+        for _ in range(max(3, args.warmup // 30)):
+            flush.fill_(1.0)
+            step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
+        for a, b in ev:
+            flush.fill_(1.0)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        rc = pa.pa_get_error(stream)
+        if rc != pa.PA_OK:
+            raise pa.PackAttnError(rc, name)
+        ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+        res[name] = {"processed_tokens": int(sum(lay["segments"])), "real_tokens": int(sum(real)),
+                     "token_utilisation": lay["token_utilisation"], "ms_fwd_bwd": ms,
+                     "valid_tflops_fwd_bwd": 3.5 * valid / (ms * 1e-3) / 1e12}
+    base = res["padded"]["ms_fwd_bwd"]
+    for r in res.values():
+        r["relative_throughput"] = base / r["ms_fwd_bwd"]
+    print(json.dumps({"study": "padded vs bucketed (groups of 4) vs packed: forward + backward attention",
+                      "workload": workload_desc(cfg)["workload"], "heads": H, "head_dim": d,
+                      "valid_flops_fwd_bwd": 3.5 * valid, "schemes": res,
+                      "pages_table_a100": {"padded": [0.45, 1.0], "bucketed": [0.78, 1.3], "packed": [0.97, 2.1]},
+                      "note": "the pages' figures are whole training throughput on an A100, for context only"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -468,12 +529,16 @@ def main():
     ap.add_argument("--config", default="mixed", choices=workloads.CONFIG_NAMES)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--packing-study", action="store_true",
+                    help="padded vs bucketed vs packed layouts of the training image mix (one GPU)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.packing_study:
+            return run_packing_study(args, local)
         return run_ours(args, world, rank, local)
     finally:
         if world > 1:

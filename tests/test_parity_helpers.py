@@ -24,3 +24,14 @@ def test_bound_is_stated_value_below_two_and_one_ulp_above():
     lse = np.zeros(3)
     assert parity.errors(ok, lse, ref, lse)["bound_ratio"] <= 1.0
     assert parity.errors(bad, lse, ref, lse)["bound_ratio"] > 1.0
+
+
+def test_packing_layouts():
+    import workloads
+    lays = workloads.packing_layouts([100, 400, 250, 0, 50, 300], bucket_size=2)
+    assert lays["packed"]["segments"] == [100, 400, 250, 50, 300]
+    assert lays["padded"]["segments"] == [400] * 5
+    assert lays["bucketed"]["segments"] == [100, 100, 300, 300, 400]  # sorted 50,100 | 250,300 | 400
+    assert abs(lays["padded"]["token_utilisation"] - 1100 / 2000) < 1e-12
+    assert abs(lays["bucketed"]["token_utilisation"] - 1100 / 1200) < 1e-12
+    assert lays["packed"]["token_utilisation"] == 1.0

@@ -104,6 +104,31 @@ def sampled_rows(cfg, per_head=None):
     return torch.cat(toks), torch.cat(heads)
 
 
+def packing_layouts(lengths, bucket_size=4):
+    """The same image mix laid out three ways (Mage-Flow page, the table after "Packing +
+    Flash Attention varlen": padding to the longest, bucket grouping, native packing).
+
+    Returns {scheme: dict(segments=[...], token_utilisation=u)} where ``segments`` are the
+    sequence lengths a kernel processes: every image padded to the longest ("padded");
+    images sorted by length and cut into groups of ``bucket_size``, each padded to its
+    group's longest ("bucketed"); the images as they are ("packed").  The token
+    utilisation is real tokens / processed tokens.
+    """
+    lengths = [int(n) for n in lengths if int(n) > 0]
+    real = sum(lengths)
+    longest = max(lengths)
+    padded = [longest] * len(lengths)
+    srt = sorted(lengths)
+    bucketed = []
+    for i in range(0, len(srt), bucket_size):
+        grp = srt[i:i + bucket_size]
+        bucketed += [max(grp)] * len(grp)
+    out = {}
+    for name, segs in (("padded", padded), ("bucketed", bucketed), ("packed", list(lengths))):
+        out[name] = dict(segments=segs, token_utilisation=real / float(sum(segs)))
+    return out
+
+
 def random_dout(shape, seed):
     """The upstream gradient dL/dout of a backward workload: N(0,1) in fp32 from its own
     seeded CPU generator, rounded to bf16."""
