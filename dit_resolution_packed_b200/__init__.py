@@ -60,6 +60,10 @@ def load_library(path=None):
     lib.pa_varlen_attn_bwd.restype = ctypes.c_int
     lib.pa_varlen_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float,
                                        vp, vp, vp, vp]
+    lib.pa_qkv_rope_fwd.restype = ctypes.c_int
+    lib.pa_qkv_rope_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp]
+    lib.pa_linear_fwd.restype = ctypes.c_int
+    lib.pa_linear_fwd.argtypes = [vp, vp, i32, i32, i32, vp, vp]
     lib.pa_get_error.restype = ctypes.c_int
     lib.pa_get_error.argtypes = [vp]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -197,6 +201,58 @@ def varlen_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, max_seqlen, scale=None,
     if rc != PA_OK:
         raise PackAttnError(rc, "pa_varlen_attn_bwd")
     return dq, dk, dv
+
+
+def _check_bf16(**tensors):
+    import torch
+    for name, t in tensors.items():
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def pa_qkv_rope_fwd(x, w_qkv, cu_seqlens, max_seqlen, rope_theta, q, k, v, stream=None):
+    """C ``pa_qkv_rope_fwd``: x [T, C], w_qkv [3*H*d, C], q, k, v [T, H, d] (bf16); cu_seqlens int32 [B+1]."""
+    _check_bf16(x=x, w_qkv=w_qkv, q=q, k=k, v=v)
+    T, C = x.shape
+    _, H, d = q.shape
+    if w_qkv.shape != (3 * H * d, C) or k.shape != q.shape or v.shape != q.shape or q.shape[0] != T:
+        raise ValueError("shape mismatch: x [T, C], w_qkv [3*H*d, C], q, k, v [T, H, d]")
+    B = cu_seqlens.numel() - 1
+    return load_library().pa_qkv_rope_fwd(_ptr(x), _ptr(w_qkv), _ptr(cu_seqlens), B, T, C, H, d, int(max_seqlen),
+                                          float(rope_theta), _ptr(q), _ptr(k), _ptr(v), _stream_handle(stream))
+
+
+def qkv_rope_fwd(x, w_qkv, cu_seqlens, max_seqlen, heads, head_dim, rope_theta=10000.0, stream=None):
+    """Fused QKV projection + RoPE; returns q, k, v bf16 [T, H, d]."""
+    import torch
+    T = x.shape[0]
+    q, k, v = (torch.empty(T, heads, head_dim, dtype=torch.bfloat16, device=x.device) for _ in range(3))
+    rc = pa_qkv_rope_fwd(x, w_qkv, cu_seqlens, max_seqlen, rope_theta, q, k, v, stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_qkv_rope_fwd")
+    return q, k, v
+
+
+def pa_linear_fwd(x, w, y, stream=None):
+    """C ``pa_linear_fwd``: y [rows, out] = x [rows, in] w[out, in]^T (bf16)."""
+    _check_bf16(x=x, w=w, y=y)
+    rows, fin = x.shape
+    fout = w.shape[0]
+    if w.shape != (fout, fin) or y.shape != (rows, fout):
+        raise ValueError("shape mismatch: x [rows, in], w [out, in], y [rows, out]")
+    return load_library().pa_linear_fwd(_ptr(x), _ptr(w), rows, fin, fout, _ptr(y), _stream_handle(stream))
+
+
+def linear_fwd(x, w, stream=None):
+    """y = x w^T (bf16) through ``pa_linear_fwd``."""
+    import torch
+    y = torch.empty(x.shape[0], w.shape[0], dtype=torch.bfloat16, device=x.device)
+    rc = pa_linear_fwd(x, w, y, stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_linear_fwd")
+    return y
 
 
 def pa_get_error(stream=None):

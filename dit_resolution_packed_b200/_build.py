@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpackattn.so")
 SOURCES = ["packattn.cu"]
-HEADERS = ["sm100_ptx.cuh", "schedule.cuh", "attn_fwd_sm100.cuh", "attn_bwd_sm100.cuh", "exp2_poly.cuh"]
+HEADERS = ["sm100_ptx.cuh", "schedule.cuh", "attn_fwd_sm100.cuh", "attn_bwd_sm100.cuh", "gemm_sm100.cuh", "exp2_poly.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -17,6 +17,7 @@
 
 #include "attn_bwd_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
+#include "gemm_sm100.cuh"
 #include "packattn.h"
 #include "schedule.cuh"
 
@@ -50,6 +51,10 @@ struct StreamState {
   int32_t* status = nullptr;  // never moves once allocated
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
+  // rotary-embedding table of the last QKV projection: (cos, sin) [rope_rows][rope_d/2]
+  float2* rope = nullptr;
+  int32_t rope_rows = 0, rope_d = 0;
+  double rope_theta = 0.0;
 };
 
 std::mutex g_mu;
@@ -129,6 +134,12 @@ int ensure_device(int device) {
   if (cudaFuncSetAttribute(pa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            pa::FwdCfg<128>::kSmemBytes) != cudaSuccess)
     return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::gemm_kernel<pa::kEpiPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::kGemmSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::gemm_kernel<pa::kEpiQkvRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::kGemmSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
   if (cudaFuncSetAttribute(pa::attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            pa::BwdCfg<64>::kSmemBytes) != cudaSuccess)
     return PA_ERR_CUDA;
@@ -152,6 +163,29 @@ bool encode_map(CUtensorMap* m, const void* base, int32_t rows, int32_t heads, i
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// A bf16 row-major [outer, inner] matrix, box {64, box_outer}, 128-byte swizzle.
+bool encode_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * 2};
+  const cuuint32_t box[2] = {64, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launches the projection GEMM (epilogue kEpi) on the persistent grid.
+template <int kEpi>
+int launch_gemm(const pa::GemmParams& gp, int dev, cudaStream_t stream) {
+  const int64_t tiles = ((static_cast<int64_t>(gp.M) + pa::kGemmBM - 1) / pa::kGemmBM) *
+                        ((static_cast<int64_t>(gp.N) + pa::kGemmBN - 1) / pa::kGemmBN);
+  const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, tiles));
+  pa::gemm_kernel<kEpi><<<grid, pa::kGemmThreads, pa::kGemmSmemBytes, stream>>>(gp);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 // Backward workspace: the schedule, then lse * log2(e) and D head-major [H][T],
 // then the fp32 dq accumulator [H][d/4][T] x 4.
@@ -443,6 +477,113 @@ int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* 
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+int pa_linear_fwd(const void* x, const void* w, int32_t rows, int32_t in_features, int32_t out_features, void* y,
+                  void* stream_handle) {
+  if (rows < 0 || in_features < 1 || out_features < 1) return PA_ERR_SHAPE;
+  if (in_features % 8 != 0 || out_features % 32 != 0) return PA_ERR_SHAPE;
+  if (rows == 0) return PA_OK;
+  if (!x || !w || !y) return PA_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16)) return PA_ERR_ALIGN;
+  int dev = -1, d2 = -1, rc;
+  if ((rc = device_of(x, &dev)) != PA_OK) return rc;
+  for (const void* ptr : {w, static_cast<const void*>(y)}) {
+    if ((rc = device_of(ptr, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  pa::GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  if (!encode_2d(&gp.tm_a, x, in_features, rows, 128) || !encode_2d(&gp.tm_b, w, in_features, out_features, 256))
+    return PA_ERR_CUDA;
+  gp.M = rows;
+  gp.N = out_features;
+  gp.K = in_features;
+  gp.y = y;
+  gp.status = st->status;
+  gp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  gp.err_timeout = PA_ERR_TIMEOUT;
+  return launch_gemm<pa::kEpiPlain>(gp, dev, stream);
+}
+
+int pa_qkv_rope_fwd(const void* x, const void* w_qkv, const int32_t* cu_seqlens, int32_t batch,
+                    int32_t total_tokens, int32_t hidden, int32_t heads, int32_t head_dim, int32_t max_seqlen,
+                    float rope_theta, void* q, void* k, void* v, void* stream_handle) {
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0 || hidden < 1 || hidden % 8 != 0) return PA_ERR_SHAPE;
+  if (!std::isfinite(rope_theta)) return PA_ERR_SCALE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  const bool rotate = rope_theta > 0.f;
+  if (rotate && max_seqlen < 1) return PA_ERR_MAX_SEQLEN;
+  if (static_cast<int64_t>(heads) * head_dim * 3 >= (int64_t(1) << 30)) return PA_ERR_SHAPE;
+  if (!x || !w_qkv || !q || !k || !v || (rotate && !cu_seqlens)) return PA_ERR_NULL;
+  const void* a16[5] = {x, w_qkv, q, k, v};
+  for (const void* ptr : a16)
+    if (!aligned(ptr, 16)) return PA_ERR_ALIGN;
+  if (rotate && !aligned(cu_seqlens, 4)) return PA_ERR_ALIGN;
+  int dev = -1, d2 = -1, rc;
+  if ((rc = device_of(x, &dev)) != PA_OK) return rc;
+  for (const void* ptr : {w_qkv, static_cast<const void*>(q), static_cast<const void*>(k),
+                          static_cast<const void*>(v), static_cast<const void*>(cu_seqlens)}) {
+    if (ptr == nullptr) continue;
+    if ((rc = device_of(ptr, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  const int32_t N = 3 * heads * head_dim;
+  pa::GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  if (!encode_2d(&gp.tm_a, x, hidden, total_tokens, 128) || !encode_2d(&gp.tm_b, w_qkv, hidden, N, 256))
+    return PA_ERR_CUDA;
+  if (rotate) {
+    // positions in the workspace; the (cos, sin) table cached per (device, stream)
+    if ((rc = ensure_workspace(st, 4 * static_cast<size_t>(total_tokens))) != PA_OK) return rc;
+    if (st->rope == nullptr || st->rope_rows < max_seqlen || st->rope_d != head_dim ||
+        st->rope_theta != static_cast<double>(rope_theta)) {
+      if (st->rope) cudaFreeAsync(st->rope, stream);
+      st->rope = nullptr;
+      const size_t n = static_cast<size_t>(max_seqlen) * (head_dim / 2);
+      if (cudaMallocAsync(reinterpret_cast<void**>(&st->rope), n * sizeof(float2), stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+      pa::rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+          st->rope, max_seqlen, head_dim, static_cast<double>(rope_theta));
+      if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+      st->rope_rows = max_seqlen;
+      st->rope_d = head_dim;
+      st->rope_theta = static_cast<double>(rope_theta);
+    }
+    int32_t* pos = reinterpret_cast<int32_t*>(st->ws);
+    pa::rope_positions_kernel<<<static_cast<unsigned>((total_tokens + 255) / 256), 256, 0, stream>>>(
+        cu_seqlens, batch, total_tokens, max_seqlen, st->rope_rows, pos, st->status, PA_ERR_CU_SEQLENS,
+        PA_ERR_MAX_SEQLEN);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    gp.pos = pos;
+    gp.rope = st->rope;
+  }
+  gp.M = total_tokens;
+  gp.N = N;
+  gp.K = hidden;
+  gp.q = q;
+  gp.k = k;
+  gp.v = v;
+  gp.heads = heads;
+  gp.head_dim = head_dim;
+  gp.status = st->status;
+  gp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  gp.err_timeout = PA_ERR_TIMEOUT;
+  return launch_gemm<pa::kEpiQkvRope>(gp, dev, stream);
+}
+
 int pa_get_error(void* stream_handle) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
   std::lock_guard<std::mutex> lock(g_mu);
@@ -490,6 +631,7 @@ void pa_release_workspace(void) {
     if (cudaSetDevice(s->device) == cudaSuccess) {
       cudaDeviceSynchronize();
       if (s->ws) cudaFree(s->ws);
+      if (s->rope) cudaFree(s->rope);
       if (s->status) cudaFree(s->status);
     }
     delete s;

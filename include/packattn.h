@@ -118,6 +118,47 @@ PA_API int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const
                               void* dv, void* stream);
 
 /*
+ * pa_qkv_rope_fwd -- the fused QKV projection in front of the attention (Mage-Flow
+ * page, "DiT Block" data flow: x -> [Q,K,V] projection -> RoPE -> attention, and
+ * "fusion strategy one": one GEMM with the stacked weight, its output split into
+ * q, k, v), enqueued on `stream`:
+ *     qkv = x W_qkv^T;  q, k, v = the [T, H, d] slices of qkv (rows of W_qkv: the
+ *     H*d rows of q, then of k, then of v, head-major);
+ *     q, k rotated by the rotary embedding (rotate-half pairs (c, c + d/2),
+ *     theta_i = rope_theta^(-2i/d)) at each token's position inside its own image.
+ *
+ *   x            device, bf16, [total_tokens, hidden], row-major, 16-byte aligned.
+ *   w_qkv        device, bf16, [3 * heads * head_dim, hidden], row-major (the
+ *                layout of a linear layer's weight), 16-byte aligned.
+ *   cu_seqlens   device, int32, [batch + 1], as for pa_varlen_attn_fwd (only read
+ *                when rope_theta > 0; positions restart at every segment).
+ *   hidden       C, a multiple of 8.   heads H >= 1.   head_dim d in {64, 128}.
+ *   max_seqlen   an upper bound of every segment length (>= 1 when rotating).
+ *   rope_theta   base of the rotary frequencies; <= 0 disables the rotation.
+ *   q, k, v      device, bf16, [total_tokens, heads, head_dim], 16-byte aligned,
+ *                written (rounded once to nearest even after the rotation).
+ *
+ * Workspace: token positions in the (device, stream) workspace and a table of
+ * (cos, sin) per (position, frequency), computed in fp64 and kept per (device,
+ * stream) until max_seqlen grows or head_dim / rope_theta change.  Errors: as for
+ * pa_varlen_attn_fwd; invalid cu_seqlens or a segment longer than max_seqlen are
+ * recorded in the status word (pa_get_error).
+ */
+PA_API int pa_qkv_rope_fwd(const void* x, const void* w_qkv, const int32_t* cu_seqlens, int32_t batch,
+                           int32_t total_tokens, int32_t hidden, int32_t heads, int32_t head_dim,
+                           int32_t max_seqlen, float rope_theta, void* q, void* k, void* v, void* stream);
+
+/*
+ * pa_linear_fwd -- y = x W^T on `stream` (the attention's output projection,
+ * Mage-Flow page, "DiT Block" data flow: attention -> output projection).
+ *   x [rows, in_features], W [out_features, in_features], y [rows, out_features]:
+ *   device, bf16, row-major, 16-byte aligned; in_features a multiple of 8,
+ *   out_features a multiple of 32.  fp32 accumulation, y rounded once.
+ */
+PA_API int pa_linear_fwd(const void* x, const void* w, int32_t rows, int32_t in_features, int32_t out_features,
+                         void* y, void* stream);
+
+/*
  * pa_get_error -- synchronise `stream`, return the first device-side error
  * recorded for the calling device and `stream` since the last call (PA_OK if
  * none) and clear it.  Returns PA_ERR_CUDA if the synchronisation fails.

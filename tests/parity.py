@@ -85,3 +85,30 @@ def bwd_check(errs, name=""):
     assert errs["finite"], (name, errs)
     assert errs["rel_fro"] <= BWD_REL_FRO, (name, errs)
     assert errs["max_abs"] <= BWD_MAX_REL * errs["ref_max"] + 1e-30, (name, errs)
+
+
+# ---- projections (pa_qkv_rope_fwd, pa_linear_fwd) against the fp64 projection oracle
+#
+# bf16 x bf16 products are exact in fp32 and the fp32 sums over the hidden size add
+# errors far below bf16's resolution; the rotation uses fp32 (cos, sin) rounded from
+# fp64; the output is rounded to bf16 once (half an ulp: 2^-9 relative).  Bound per
+# element: 2^-8 |ref| (twice the rounding) + 1e-4 rms(ref) for outputs near zero;
+# relative Frobenius error <= 2e-3.
+PROJ_REL = 2.0 ** -8
+PROJ_ABS_RMS = 1e-4
+PROJ_REL_FRO = 2e-3
+
+
+def proj_check(got, ref, name=""):
+    g = np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    d = np.abs(g - r)
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    bound = PROJ_REL * np.abs(r) + PROJ_ABS_RMS * rms
+    worst = float(np.max(d / np.maximum(bound, 1e-300))) if r.size else 0.0
+    rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
+    errs = dict(worst_over_bound=worst, rel_fro=rel, finite=bool(np.all(np.isfinite(g))))
+    assert errs["finite"], (name, errs)
+    assert worst <= 1.0, (name, errs)
+    assert rel <= PROJ_REL_FRO, (name, errs)
+    return errs

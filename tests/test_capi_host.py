@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 11
+    assert len(names) == len(set(names)) == 13
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -93,6 +93,25 @@ def test_bwd_host_validation_before_any_cuda_call(lib):
     assert raw(dq=24) == pa.PA_ERR_ALIGN
     assert raw(out=8) == pa.PA_ERR_ALIGN
     assert raw(lse=18) == pa.PA_ERR_ALIGN
+
+
+def test_projection_host_validation_before_any_cuda_call(lib):
+    f = lib.pa_linear_fwd
+    assert f(16, 16, 4, 12, 64, 16, None) == pa.PA_ERR_SHAPE       # in_features not a multiple of 8
+    assert f(16, 16, 4, 16, 48, 16, None) == pa.PA_ERR_SHAPE       # out_features not a multiple of 32
+    assert f(16, 16, 0, 16, 64, 16, None) == pa.PA_OK
+    assert f(None, 16, 4, 16, 64, 16, None) == pa.PA_ERR_NULL
+    assert f(16, 24, 4, 16, 64, 16, None) == pa.PA_ERR_ALIGN
+    g = lib.pa_qkv_rope_fwd
+    args = lambda **kw: (kw.get("x", 16), 16, kw.get("cu", 16), kw.get("batch", 1), kw.get("total", 4),
+                         kw.get("hidden", 64), 1, kw.get("d", 64), kw.get("max_seqlen", 4),
+                         ctypes.c_float(kw.get("theta", 10000.0)), 16, 16, 16, None)
+    assert g(*args(d=96)) == pa.PA_ERR_HEAD_DIM
+    assert g(*args(hidden=60)) == pa.PA_ERR_SHAPE
+    assert g(*args(theta=math.nan)) == pa.PA_ERR_SCALE
+    assert g(*args(max_seqlen=0)) == pa.PA_ERR_MAX_SEQLEN
+    assert g(*args(cu=None)) == pa.PA_ERR_NULL
+    assert g(*args(batch=0, total=0)) == pa.PA_OK
 
 
 def test_missing_library_fails_loudly(tmp_path):
