@@ -337,6 +337,39 @@ def run_ours(args, world, rank, local):
     bwd_ms = allreduce_max(sum(bwd_step_ms), world, device) / args.steps
     bq10, bq50, bq90 = (float(x) for x in np.percentile(bwd_step_ms, [10, 50, 90]))
 
+    # ---- the projections around the attention at this pack's shape (hidden = H*d): the fused
+    # QKV projection with RoPE and the output projection, on synthetic x and weights
+    C = H * d
+    px = workloads.random_dout((T, C), 31 + rank).to(device)
+    pw = (workloads.random_dout((3 * H * d, C), 32).float() * C ** -0.5).to(torch.bfloat16).to(device)
+    pwo = (workloads.random_dout((C, H * d), 33).float() * (H * d) ** -0.5).to(torch.bfloat16).to(device)
+    pq, pk, pv = (torch.empty(T, H, d, dtype=torch.bfloat16, device=device) for _ in range(3))
+    py = torch.empty(T, C, dtype=torch.bfloat16, device=device)
+    o2 = out.view(T, H * d)
+
+    def proj_time(fn):
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.fill_(1.0)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return allreduce_max(sum(a.elapsed_time(b) for a, b in evs), world, device) / args.steps
+
+    qkv_ms = proj_time(lambda: pa.pa_qkv_rope_fwd(px, pw, cu, p["max_seqlen"], 10000.0, pq, pk, pv, stream))
+    out_ms = proj_time(lambda: pa.pa_linear_fwd(o2, pwo, py, stream))
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, "projections")
+    qkv_flops, out_flops = 2.0 * T * C * 3 * H * d, 2.0 * T * H * d * C
+
     # ---- end to end through the public API with host buffers (pinned): every step copies its
     # q, k, v, cu_seqlens host -> device and its out, lse device -> host inside the timed region.
     # Steps are pipelined the way an input pipeline runs them: two device buffer sets and three
@@ -446,6 +479,13 @@ def run_ours(args, world, rank, local):
                          "frac": bwd_flops / (bkern_ms_total / max(1, bkern_n) * 1e-3) / 1e12 / bpeak,
                          "peak_source": bpeak_src, "traffic": None},
             "gpu_launches": 4 * args.steps,  # prep, schedule, main, dq conversion per step
+        },
+        "projections": {
+            "hidden": C, "note": "synthetic x and weights at this pack's shape; same steps, warm-up and L2 flush",
+            "qkv_rope": {"value": qkv_flops * world / (qkv_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": qkv_ms,
+                         "flops_per_step": qkv_flops, "kernel": "gemm_kernel<QKV+RoPE>"},
+            "out_proj": {"value": out_flops * world / (out_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": out_ms,
+                         "flops_per_step": out_flops, "kernel": "gemm_kernel<plain>"},
         },
         "gpu_launches": 2 * args.steps,  # schedule + attention kernel per step, headline timed region
         "clocks": clock_rec,
