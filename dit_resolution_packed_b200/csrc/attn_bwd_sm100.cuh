@@ -66,9 +66,12 @@ struct BwdCfg {
   static constexpr int kOffBar = kOffStage + 2 * 128 * 4;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + 1024 for base alignment
   static constexpr uint32_t kTmemCols = 512;
-  // tensor memory: A [0,128) S^T then P^T; B [128,256) dP^T, dS^T, then dQ;
-  // dV [256, 256+d); dK [256+d, 256+2d)
+  // tensor memory: A [0,128) S^T then P^T; B [128,256) dP^T, dS^T (and dQ at d = 128);
+  // dV [256, 256+d); dK [256+d, 256+2d); at d = 64 dQ has its own columns [384, 448),
+  // so the next dP^T does not wait for the read-out of the last dQ.
+  static constexpr bool kOwnDq = 256 + 3 * D <= 512;
   static constexpr uint32_t kColA = 0, kColB = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr uint32_t kColDQ = kOwnDq ? 256 + 2 * D : kColB;
 };
 
 struct BwdParams {
@@ -292,7 +295,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
     bwd_issue_kmajor<D>(leader, tmem + C::kColA, k_addr, q_addr0 + qslot * C::kTileBytes);
     for (int32_t i = 0; i < w.nq; ++i) {
       const int cur = qslot;
-      if (dq_pending) {  // tensor memory B: the previous dQ partial has been read
+      if (!C::kOwnDq && dq_pending) {  // tensor memory B: the previous dQ partial has been read
         if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
         dqe_ph ^= 1u;
         tc_fence_after();
@@ -309,8 +312,13 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
       }
       bwd_issue_tmem_a<D>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
       bwd_issue_tmem_a<D>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
+      if (C::kOwnDq && dq_pending) {  // dQ's own columns: the previous partial has been read
+        if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
+        dqe_ph ^= 1u;
+        tc_fence_after();
+      }
       // dQ before the next S^T, so that its read-out overlaps that MMA
-      bwd_issue_dq<D>(leader, tmem + C::kColB, ds_addr, k_addr);
+      bwd_issue_dq<D>(leader, tmem + C::kColDQ, ds_addr, k_addr);
       mma_commit_if(leader, &bars->dq_full);
       dq_pending = true;
       mma_commit_if(leader, &bars->qd_empty[cur]);
@@ -441,7 +449,7 @@ __device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* ba
   const int t = threadIdx.x & 127;
   const int lane = threadIdx.x & 31;
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
-  const uint32_t tB = tmem + lane_base + C::kColB;
+  const uint32_t tB = tmem + lane_base + C::kColDQ;  // the dQ partial
   const uint32_t tDV = tmem + lane_base + C::kColDV;
   const uint32_t tDK = tmem + lane_base + C::kColDK;
   uint32_t sk = 0, dqf_ph = 0, dkvf_ph = 0;

@@ -95,3 +95,24 @@ def test_bwd_device_rejects_bad_cu_seqlens(cuda_device):
     assert rc == pa.PA_OK
     assert pa.pa_get_error() == pa.PA_ERR_CU_SEQLENS
     _full_check(p, cuda_device)
+
+
+@pytest.mark.parametrize("name,per_head", [("long", 6), ("interactive", 3)])
+def test_bwd_full_size_sampled_dq_rows_and_closed_forms(cuda_device, name, per_head):
+    """Full-size packs (65 536 tokens at d = 64; 16 384 tokens with outlier keys at d = 128):
+    dq of sampled query rows against the oracle, and per head the closed forms of the exact
+    gradient, sum_j dv_j = sum_r dout_r and sum_j dk_j = 0, within the accumulated bf16 rounding."""
+    cfg = workloads.load_config(name)
+    p = workloads.make_inputs(cfg)
+    dq, dk, dv, dout, sc = _forward_backward(p, cuda_device, 51)
+    tok, head = workloads.sampled_rows(cfg, per_head=per_head)
+    ref = oracle.varlen_attention_bwd(p["q"], p["k"], p["v"], dout, p["cu_seqlens"], sc,
+                                      rows=(tok.numpy(), head.numpy()))
+    got = dq[tok.to(cuda_device), head.to(cuda_device).long()].double().cpu().numpy()
+    parity.bwd_check(parity.bwd_errors(got, ref), "dq")
+    g = dout.to(cuda_device).double()
+    for h in range(cfg["heads"]):  # one segment per pack
+        sv = dv[:, h].double().sum(0) - g[:, h].sum(0)
+        assert sv.abs().max().item() <= parity.BWD_REL_FRO * g[:, h].abs().sum(0).max().item()
+        sk = dk[:, h].double().sum(0)
+        assert sk.abs().max().item() <= parity.BWD_REL_FRO * dk[:, h].double().abs().sum(0).max().item()
