@@ -9,9 +9,8 @@
 // Tiles of 128 x 256 outputs; K in blocks of 64 (one 128-byte swizzle row) through a
 // four-stage TMA ring (48 KB per stage); tcgen05 M = 128, N = 256, K = 16 MMAs into
 // one of two 256-column tensor-memory accumulators, so that the epilogue of a tile
-// overlaps the MMAs of the next.  Persistent grid, tiles taken in row-major order
-// (N fastest), so that the CTAs running at once share their x rows and read W
-// through L2.
+// overlaps the MMAs of the next.  Persistent grid, tiles taken in bands of row tiles
+// (kGemmGroupM), so that the CTAs running at once share x rows and W panels in L2.
 //
 // CTA: warps 0-3 epilogue (one thread per output row), warp 4 TMA producer, warp 5
 // tensor-memory owner and MMA issuer (whole warp, one elected lane issues).
@@ -34,6 +33,24 @@ constexpr int kGemmOffBar = kGemmStages * kGemmStageBytes;
 constexpr int kGemmSmemBytes = kGemmOffBar + 256 + 1024;  // + 1024 for base alignment
 
 enum GemmEpilogue : int { kEpiPlain = 0, kEpiQkvRope = 1 };
+
+// Tile order: bands of kGemmGroupM row tiles, each band walked N tile by N tile, so the
+// tiles running at once share a few x rows and about half of W's panels.  Measured on
+// B200 at the mixed and training shapes against plain row-major order (1): 8 gains
+// 5-6 % on the QKV GEMM and up to 2 % on the output projection; 16 is close; column-
+// major loses 15-25 % once x outgrows L2.
+constexpr int kGemmGroupM = 8;
+
+// Row and column tile of the t-th tile in that order.
+__device__ __forceinline__ void gemm_tile(int t, int tiles_m, int tiles_n, int& mt, int& nt) {
+  const int per = kGemmGroupM * tiles_n;
+  const int g = t / per;
+  const int first = g * kGemmGroupM;
+  const int size = min(kGemmGroupM, tiles_m - first);
+  const int local = t - g * per;
+  mt = first + local % size;
+  nt = local / size;
+}
 
 struct GemmParams {
   CUtensorMap tm_a;      // x [M, K] bf16, box {64, 128}, 128-byte swizzle
@@ -71,13 +88,16 @@ __device__ __forceinline__ bool gemm_drain_wait(uint64_t* bar, uint32_t parity, 
 
 __device__ __forceinline__ void gemm_producer(const GemmParams& p, uint8_t* smem, GemmBars* bars, const WaitCtl& wc) {
   const int tiles_n = (p.N + kGemmBN - 1) / kGemmBN;
-  const int tiles = ((p.M + kGemmBM - 1) / kGemmBM) * tiles_n;
+  const int tiles_m = (p.M + kGemmBM - 1) / kGemmBM;
+  const int tiles = tiles_m * tiles_n;
   const int kblocks = (p.K + kGemmBK - 1) / kGemmBK;
   int stage = 0;
   uint32_t phase = 0, armed = 0, armed_ph = 0;
   bool ok = true;
   for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-    const int m0 = (t / tiles_n) * kGemmBM, n0 = (t % tiles_n) * kGemmBN;
+    int mt, nt;
+    gemm_tile(t, tiles_m, tiles_n, mt, nt);
+    const int m0 = mt * kGemmBM, n0 = nt * kGemmBN;
     for (int kb = 0; kb < kblocks; ++kb) {
       if (!(ok = mbar_wait(&bars->empty[stage], phase ^ 1u, wc))) break;
       mbar_arrive_expect_tx(&bars->full[stage], kGemmStageBytes);
@@ -170,7 +190,8 @@ __device__ __forceinline__ void store32_bf16(uint16_t* dst, const uint32_t (&v)[
 template <int kEpi>
 __device__ __forceinline__ void gemm_epilogue(const GemmParams& p, GemmBars* bars, const WaitCtl& wc, uint32_t tmem) {
   const int tiles_n = (p.N + kGemmBN - 1) / kGemmBN;
-  const int tiles = ((p.M + kGemmBM - 1) / kGemmBM) * tiles_n;
+  const int tiles_m = (p.M + kGemmBM - 1) / kGemmBM;
+  const int tiles = tiles_m * tiles_n;
   const int r = threadIdx.x & 127;
   const int lane = threadIdx.x & 31;
   const uint32_t lane_base = static_cast<uint32_t>(r & ~31) << 16;
@@ -182,7 +203,9 @@ __device__ __forceinline__ void gemm_epilogue(const GemmParams& p, GemmBars* bar
     if (__any_sync(0xffffffffu, !ok)) break;
     af_ph ^= 1u << buf;
     tc_fence_after();
-    const int m0 = (t / tiles_n) * kGemmBM, n0 = (t % tiles_n) * kGemmBN;
+    int mt, nt;
+    gemm_tile(t, tiles_m, tiles_n, mt, nt);
+    const int m0 = mt * kGemmBM, n0 = nt * kGemmBN;
     const int row = m0 + r;
     const bool row_ok = row < p.M;
     const uint32_t tacc = tmem + lane_base + buf * kGemmBN;
