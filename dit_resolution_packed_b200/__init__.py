@@ -64,6 +64,12 @@ def load_library(path=None):
     lib.pa_qkv_rope_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp]
     lib.pa_linear_fwd.restype = ctypes.c_int
     lib.pa_linear_fwd.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.pa_fp8_vt_keys.restype = ctypes.c_int64
+    lib.pa_fp8_vt_keys.argtypes = [i32, i32]
+    lib.pa_fp8_quantize_qkv.restype = ctypes.c_int
+    lib.pa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.pa_varlen_attn_fwd_fp8.restype = ctypes.c_int
+    lib.pa_varlen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp]
     lib.pa_get_error.restype = ctypes.c_int
     lib.pa_get_error.argtypes = [vp]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -253,6 +259,87 @@ def linear_fwd(x, w, stream=None):
     if rc != PA_OK:
         raise PackAttnError(rc, "pa_linear_fwd")
     return y
+
+
+def _check_bytes(**tensors):
+    import torch
+    for name, t in tensors.items():
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise TypeError(f"{name} must be uint8 or float8_e4m3fn, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def pa_fp8_vt_keys(batch, total_tokens):
+    """C ``pa_fp8_vt_keys``: keys per row of the transposed FP8 V buffer."""
+    return int(load_library().pa_fp8_vt_keys(int(batch), int(total_tokens)))
+
+
+def pa_fp8_quantize_qkv(q, k, v, cu_seqlens, q8, k8, v8t, scales, stream=None):
+    """C ``pa_fp8_quantize_qkv``: q, k, v bf16 [T, H, 128] -> q8, k8 [T, H, 128], v8t [H*128, keys]
+    (bytes), scales fp32 [4 + H*128].  Returns the status code."""
+    import torch
+    _check_bf16(q=q, k=k, v=v)
+    _check_bytes(q8=q8, k8=k8, v8t=v8t)
+    if scales.dtype != torch.float32 or not scales.is_contiguous():
+        raise TypeError("scales must be a contiguous float32 tensor")
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    if (k.shape != q.shape or v.shape != q.shape or q8.shape != q.shape or k8.shape != q.shape
+            or tuple(v8t.shape) != (H * d, pa_fp8_vt_keys(B, T)) or scales.numel() != 4 + H * d):
+        raise ValueError("shape mismatch: q, k, v, q8, k8 [T, H, d]; v8t [H*d, keys]; scales [4 + H*d]")
+    return load_library().pa_fp8_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, T, H, d, _ptr(q8),
+                                              _ptr(k8), _ptr(v8t), _ptr(scales), _stream_handle(stream))
+
+
+def fp8_quantize_qkv(q, k, v, cu_seqlens, stream=None):
+    """Quantise q, k, v for the FP8 forward; returns a dict q8, k8, v8t (uint8) and scales (fp32)."""
+    import torch
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    dev = q.device
+    qz = dict(q8=torch.empty(T, H, d, dtype=torch.uint8, device=dev),
+              k8=torch.empty(T, H, d, dtype=torch.uint8, device=dev),
+              v8t=torch.empty(H * d, max(pa_fp8_vt_keys(B, T), 0), dtype=torch.uint8, device=dev),
+              scales=torch.empty(4 + H * d, dtype=torch.float32, device=dev))
+    rc = pa_fp8_quantize_qkv(q, k, v, cu_seqlens, qz["q8"], qz["k8"], qz["v8t"], qz["scales"], stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_fp8_quantize_qkv")
+    return qz
+
+
+def pa_varlen_attn_fwd_fp8(q8, k8, v8t, scales, cu_seqlens, max_seqlen, scale, out, lse, stream=None):
+    """C ``pa_varlen_attn_fwd_fp8`` on the quantiser's tensors; out bf16 [T, H, 128], lse fp32 [T, H]."""
+    import torch
+    _check_bytes(q8=q8, k8=k8, v8t=v8t)
+    _check_bf16(out=out)
+    if lse.dtype != torch.float32 or scales.dtype != torch.float32:
+        raise TypeError("lse and scales must be float32")
+    T, H, d = q8.shape
+    B = cu_seqlens.numel() - 1
+    if (k8.shape != q8.shape or out.shape != q8.shape or tuple(lse.shape) != (T, H)
+            or tuple(v8t.shape) != (H * d, pa_fp8_vt_keys(B, T)) or scales.numel() != 4 + H * d):
+        raise ValueError("shape mismatch: q8, k8, out [T, H, d]; v8t [H*d, keys]; lse [T, H]; scales [4 + H*d]")
+    return load_library().pa_varlen_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8t), _ptr(scales), _ptr(cu_seqlens),
+                                                 B, T, H, d, int(max_seqlen), float(scale), _ptr(out), _ptr(lse),
+                                                 _stream_handle(stream))
+
+
+def varlen_attn_fwd_fp8(qz, cu_seqlens, max_seqlen, scale=None, out=None, lse=None, stream=None):
+    """FP8 forward on a ``fp8_quantize_qkv`` result; returns (out bf16 [T, H, 128], lse fp32 [T, H])."""
+    import torch
+    q8 = qz["q8"]
+    if scale is None:
+        scale = 1.0 / math.sqrt(q8.shape[-1])
+    if out is None:
+        out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty(q8.shape[0], q8.shape[1], dtype=torch.float32, device=q8.device)
+    rc = pa_varlen_attn_fwd_fp8(q8, qz["k8"], qz["v8t"], qz["scales"], cu_seqlens, max_seqlen, scale, out, lse,
+                                stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_varlen_attn_fwd_fp8")
+    return out, lse
 
 
 def pa_get_error(stream=None):

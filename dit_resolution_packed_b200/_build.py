@@ -13,7 +13,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpackattn.so")
 SOURCES = ["packattn.cu"]
-HEADERS = ["sm100_ptx.cuh", "schedule.cuh", "attn_fwd_sm100.cuh", "attn_bwd_sm100.cuh", "gemm_sm100.cuh", "exp2_poly.cuh"]
+HEADERS = ["sm100_ptx.cuh", "schedule.cuh", "attn_fwd_sm100.cuh", "attn_fwd_fp8_sm100.cuh", "attn_bwd_sm100.cuh",
+           "gemm_sm100.cuh", "exp2_poly.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -48,7 +49,7 @@ def _check_registers(ptxas_log):
             kernel = m.group(1)
             continue
         m = re.search(r"Used (\d+) registers", line)
-        if m and kernel and ("attn_fwd_kernel" in kernel or "attn_bwd_kernel" in kernel):
+        if m and kernel and any(n in kernel for n in ("attn_fwd_kernel", "attn_fwd_fp8_kernel", "attn_bwd_kernel")):
             regs = int(m.group(1))
             if regs != LAUNCH_REGS:
                 raise RuntimeError(f"{kernel}: {regs} registers, expected {LAUNCH_REGS} for the register split")

@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "attn_bwd_sm100.cuh"
+#include "attn_fwd_fp8_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "packattn.h"
@@ -134,6 +135,9 @@ int ensure_device(int device) {
   if (cudaFuncSetAttribute(pa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            pa::FwdCfg<128>::kSmemBytes) != cudaSuccess)
     return PA_ERR_CUDA;
+  if (cudaFuncSetAttribute(pa::attn_fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           pa::Fp8Cfg::kSmemBytes) != cudaSuccess)
+    return PA_ERR_CUDA;
   if (cudaFuncSetAttribute(pa::gemm_kernel<pa::kEpiPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            pa::kGemmSmemBytes) != cudaSuccess)
     return PA_ERR_CUDA;
@@ -175,6 +179,39 @@ bool encode_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, u
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A byte matrix [outer, inner] with a row stride of `stride` bytes, box 128 x 128,
+// 128-byte swizzle (the FP8 operands).
+bool encode_u8(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int64_t fp8_vt_keys(int32_t batch, int32_t total) {
+  return 16 * ((static_cast<int64_t>(total) + 15) / 16) + 16 * static_cast<int64_t>(batch);
+}
+
+// Events around the main kernel of a call when profiling is on (ev0 recorded here).
+int prof_begin(cudaStream_t stream, cudaEvent_t* ev1) {
+  *ev1 = nullptr;
+  if (!g_prof_on) return PA_OK;
+  if (g_prof_used == g_prof_events.size()) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return PA_ERR_CUDA;
+    g_prof_events.emplace_back(a, b);
+  }
+  cudaEventRecord(g_prof_events[g_prof_used].first, stream);
+  *ev1 = g_prof_events[g_prof_used].second;
+  ++g_prof_used;
+  return PA_OK;
 }
 
 // Launches the projection GEMM (epilogue kEpi) on the persistent grid.
@@ -776,6 +813,157 @@ int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, cons
   const cudaError_t le = head_dim == 128 ? cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<128>, fp)
                                          : cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<64>, fp);
   if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+int64_t pa_fp8_vt_keys(int32_t batch, int32_t total_tokens) {
+  if (batch < 0 || total_tokens < 0) return -1;
+  return fp8_vt_keys(batch, total_tokens);
+}
+
+int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                        int32_t total_tokens, int32_t heads, int32_t head_dim, void* q8, void* k8, void* v8t,
+                        float* scales, void* stream_handle) {
+  if (head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  if (!q || !k || !v || !cu_seqlens || !q8 || !k8 || !v8t || !scales) return PA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) || !aligned(k8, 16) ||
+      !aligned(v8t, 16) || !aligned(scales, 16) || !aligned(cu_seqlens, 4))
+    return PA_ERR_ALIGN;
+  const int64_t tiles = (static_cast<int64_t>(total_tokens) + 127) / 128;
+  if (tiles > 65535 || heads > 65535 || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24) ||
+      fp8_vt_keys(batch, total_tokens) >= (int64_t(1) << 32))
+    return PA_ERR_SHAPE;
+  int dev = -1, d2 = -1;
+  int rc;
+  if ((rc = device_of(q, &dev)) != PA_OK) return rc;
+  const void* others[7] = {k, v, cu_seqlens, q8, k8, v8t, scales};
+  for (const void* p : others) {
+    if ((rc = device_of(p, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  const size_t amax_bytes = 4 * (4 + static_cast<size_t>(heads) * head_dim);
+  if ((rc = ensure_workspace(st, amax_bytes)) != PA_OK) return rc;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(st->ws);
+  if (cudaMemsetAsync(amax, 0, amax_bytes, stream) != cudaSuccess) return PA_ERR_CUDA;
+  const int32_t nch8 = heads * head_dim / 8;
+  const int gx = (nch8 + 31) / 32;
+  const int64_t gy_want = std::max<int64_t>(1, (4 * static_cast<int64_t>(g_dev[dev].sms)) / gx);
+  const int gy = static_cast<int>(std::min<int64_t>({gy_want, (static_cast<int64_t>(total_tokens) + 7) / 8, 65535}));
+  pa::fp8_amax_kernel<<<dim3(gx, gy), pa::kQuantThreads, 0, stream>>>(
+      static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), total_tokens, nch8,
+      amax);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  pa::fp8_quantize_kernel<<<dim3(heads, static_cast<unsigned>(tiles)), pa::kQuantThreads, 0, stream>>>(
+      static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, batch,
+      total_tokens, heads, amax, static_cast<uint2*>(q8), static_cast<uint2*>(k8), static_cast<uint8_t*>(v8t),
+      fp8_vt_keys(batch, total_tokens), scales);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8t, const float* scales,
+                           const int32_t* cu_seqlens, int32_t batch, int32_t total_tokens, int32_t heads,
+                           int32_t head_dim, int32_t max_seqlen, float scale, void* out, float* lse,
+                           void* stream_handle) {
+  if (head_dim != 128) return PA_ERR_HEAD_DIM;
+  if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SCALE;
+  if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
+  if (batch == 0 || total_tokens == 0) return PA_OK;
+  if (max_seqlen < 1) return PA_ERR_MAX_SEQLEN;
+  if (!q8 || !k8 || !v8t || !scales || !cu_seqlens || !out || !lse) return PA_ERR_NULL;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8t, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens, 4))
+    return PA_ERR_ALIGN;
+  const int64_t item_bound = static_cast<int64_t>(heads) * ((static_cast<int64_t>(total_tokens) + 255) / 256 + batch);
+  const int64_t vt_keys = fp8_vt_keys(batch, total_tokens);
+  if (item_bound >= (int64_t(1) << 31) || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24) ||
+      vt_keys >= (int64_t(1) << 32))
+    return PA_ERR_SHAPE;
+  int dev = -1, d2 = -1;
+  int rc;
+  if ((rc = device_of(q8, &dev)) != PA_OK) return rc;
+  const void* others[6] = {k8, v8t, scales, out, lse, cu_seqlens};
+  for (const void* p : others) {
+    if ((rc = device_of(p, &d2)) != PA_OK) return rc;
+    if (d2 != dev) return PA_ERR_NOT_DEVICE;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
+  if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  StreamState* st = state_for(dev, stream);
+  if ((rc = ensure_status(st)) != PA_OK) return rc;
+  const WsLayout L = ws_layout(batch);
+  if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
+
+  pa::SchedParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  const int64_t hd = static_cast<int64_t>(heads) * head_dim;
+  if (!encode_u8(&sp.tmpl[0], q8, hd, total_tokens, hd) || !encode_u8(&sp.tmpl[1], k8, hd, total_tokens, hd) ||
+      !encode_u8(&sp.tmpl[2], v8t, vt_keys, hd, vt_keys))
+    return PA_ERR_CUDA;
+  sp.base[0] = q8;
+  sp.base[1] = k8;
+  sp.base[2] = v8t;
+  sp.cu = cu_seqlens;
+  sp.status = st->status;
+  sp.counts = reinterpret_cast<int32_t*>(st->ws + L.counts);
+  sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
+  sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
+  sp.maps = st->ws + L.maps;
+  sp.row_bytes = static_cast<uint64_t>(hd);
+  sp.batch = batch;
+  sp.total = total_tokens;
+  sp.heads = heads;
+  sp.max_seqlen = max_seqlen;
+  sp.rows_log2 = 8;
+  sp.v_keys_inner = 1;
+  sp.err_cu = PA_ERR_CU_SEQLENS;
+  sp.err_max = PA_ERR_MAX_SEQLEN;
+  pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+
+  pa::Fp8Params fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.f.cu = cu_seqlens;
+  fp.f.out = out;
+  fp.f.lse = lse;
+  fp.f.counts = sp.counts;
+  fp.f.next_item = sp.counts + 2;
+  fp.f.order = sp.order;
+  fp.f.item_start = sp.item_start;
+  fp.f.maps = sp.maps;
+  fp.f.status = st->status;
+  fp.f.heads = heads;
+  fp.f.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  fp.f.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  fp.f.err_timeout = PA_ERR_TIMEOUT;
+  fp.scales = scales;
+  const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
+  cudaEvent_t ev1 = nullptr;
+  if ((rc = prof_begin(stream, &ev1)) != PA_OK) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.dynamicSmemBytes = pa::Fp8Cfg::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = g_prof_on ? 0 : 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pa::attn_fwd_fp8_kernel, fp) != cudaSuccess || cudaGetLastError() != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (ev1) cudaEventRecord(ev1, stream);
   return PA_OK;
 }
 

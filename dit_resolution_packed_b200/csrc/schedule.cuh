@@ -15,7 +15,8 @@
 //   4. for the forward, writes three tensor maps per segment (q, k, v) whose
 //      base is the segment's first token and whose row extent is L, so that
 //      every TMA tile stops at the segment boundary: loads past it read zeros
-//      and no tile touches another image (maps == nullptr skips this step).
+//      and no tile touches another image (maps == nullptr skips this step);
+//      the FP8 variant's transposed V map is cut along its key axis instead.
 //
 // The mask of the method (Mage-Flow page, "Packing + Flash Attention varlen":
 // images attend only to themselves, no padding) is thereby carried entirely by
@@ -45,6 +46,10 @@ struct SchedParams {
   uint64_t row_bytes;      // H * d * 2
   int32_t batch, total, heads, max_seqlen;
   int32_t rows_log2;        // rows of a work item: 2^rows_log2 (8 forward, 7 backward)
+  // nonzero: the third map (v) is over a [channels][keys] matrix whose segment s
+  // starts at key 16*ceil(cu[s]/16) + 16*s (the FP8 variant's transposed V); its
+  // per-segment map moves the base to that key and sets the key extent to L
+  int32_t v_keys_inner;
   int32_t err_cu, err_max;  // status codes to record
 };
 
@@ -135,6 +140,12 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     const uint4* src = reinterpret_cast<const uint4*>(&p.tmpl[which]);
 #pragma unroll
     for (int w = 0; w < 8; ++w) reinterpret_cast<uint4*>(dst)[w] = src[w];
+    if (which == 2 && p.v_keys_inner) {
+      const uint64_t key0 = 16ull * ((static_cast<uint64_t>(beg) + 15) / 16) + 16ull * static_cast<uint64_t>(s);
+      tmap_replace_address(dst, static_cast<const uint8_t*>(p.base[2]) + key0);
+      tmap_replace_dim0(dst, static_cast<uint32_t>(len));
+      continue;
+    }
     const uint8_t* seg_base = static_cast<const uint8_t*>(p.base[which]) + static_cast<uint64_t>(beg) * p.row_bytes;
     tmap_replace_address(dst, seg_base);
     tmap_replace_dim1(dst, static_cast<uint32_t>(len));

@@ -120,6 +120,12 @@ __device__ __forceinline__ void tmap_replace_dim1(void* gmap, uint32_t extent) {
                "r"(extent)
                : "memory");
 }
+__device__ __forceinline__ void tmap_replace_dim0(void* gmap, uint32_t extent) {
+  asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 0, %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(gmap)),
+               "r"(extent)
+               : "memory");
+}
 __device__ __forceinline__ void fence_tmap_release() {
   asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
 }

@@ -159,6 +159,61 @@ PA_API int pa_linear_fwd(const void* x, const void* w, int32_t rows, int32_t in_
                          void* y, void* stream);
 
 /*
+ * FP8 (E4M3) variant of the forward, head_dim 128 (FPS Attention slides of the
+ * Mage-Flow talk: attention on FP8 operands with Q and K quantised per tensor, V per
+ * channel and the softmax weights P per tensor).  Two calls: the quantiser, then the
+ * attention on its output.
+ *
+ * pa_fp8_vt_keys -- keys per row of the transposed V buffer for a pack of `batch`
+ * segments and `total_tokens` tokens: 16*ceil(total_tokens/16) + 16*batch (-1 if
+ * an argument is negative).  Segment s of the pack occupies keys
+ * [16*ceil(cu[s]/16) + 16*s, + L_s) of every row, so that each starts on a
+ * 16-byte boundary (the TMA copy rule); the keys between segments are never read.
+ */
+PA_API int64_t pa_fp8_vt_keys(int32_t batch, int32_t total_tokens);
+
+/*
+ * pa_fp8_quantize_qkv -- quantise bf16 q, k, v to E4M3 on `stream`.
+ *   q, k, v      device, bf16, [total_tokens, heads, 128], 16-byte aligned (read).
+ *   cu_seqlens   device, int32, [batch + 1], as for pa_varlen_attn_fwd (the layout
+ *                of v8t depends on it; it is not validated here).
+ *   q8, k8       device, [total_tokens, heads, 128] bytes, 16-byte aligned (written).
+ *   v8t          device, [heads*128][pa_fp8_vt_keys(batch, total_tokens)] bytes,
+ *                16-byte aligned: v8 transposed per (head, channel) row, segment
+ *                by segment as pa_fp8_vt_keys describes (only the segments' keys
+ *                are written).
+ *   scales       device, fp32, [4 + heads*128], 16-byte aligned (written):
+ *                [0] s_q, [1] s_k, [2..3] zero, [4 + h*128 + c] s_v of (h, c).
+ * With a = the absolute maximum of a group (the whole q; the whole k; the column
+ * (h, c) of v over all tokens): mult = 448 / a, s = a / 448 (fp32, correctly
+ * rounded; both 1 when a = 0) and code = E4M3(fp32(x * mult)), rounded to nearest
+ * even and clamped to +-448.  x = s * value(code) is the dequantised input.
+ * Workspace: the absolute maxima, in the (device, stream) workspace.  Errors:
+ * PA_ERR_HEAD_DIM unless head_dim = 128; otherwise as for pa_varlen_attn_fwd.
+ * Inputs with NaN give undefined codes.
+ */
+PA_API int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                               int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim, void* q8,
+                               void* k8, void* v8t, float* scales, void* stream);
+
+/*
+ * pa_varlen_attn_fwd_fp8 -- the packed varlen attention forward on the quantiser's
+ * output (q8, k8, v8t, scales as pa_fp8_quantize_qkv writes them; the same pack,
+ * heads and cu_seqlens).  Computes, with x = scale * s_q * s_k * (q8 . k8) per key,
+ *     out[r,h,c] = s_v[h,c] * sum_j P8_j v8[j,h,c] / sum_j P8_j,
+ *     lse[r,h]   = log sum_j exp(x_j),
+ * where P8_j is E4M3 of exp(x_j - m) times a power of two (m: a running maximum of
+ * the row), i.e. softmax weights rounded to E4M3 relative to the row's largest
+ * ones.  out bf16 [total_tokens, heads, 128], lse fp32 [total_tokens, heads] as for
+ * pa_varlen_attn_fwd; other arguments, ownership, workspace and errors likewise
+ * (PA_ERR_HEAD_DIM unless head_dim = 128; q8, k8, v8t, scales 16-byte aligned).
+ */
+PA_API int pa_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8t, const float* scales,
+                                  const int32_t* cu_seqlens, int32_t batch, int32_t total_tokens, int32_t heads,
+                                  int32_t head_dim, int32_t max_seqlen, float scale, void* out, float* lse,
+                                  void* stream);
+
+/*
  * pa_get_error -- synchronise `stream`, return the first device-side error
  * recorded for the calling device and `stream` since the last call (PA_OK if
  * none) and clear it.  Returns PA_ERR_CUDA if the synchronisation fails.

@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 13
+    assert len(names) == len(set(names)) == 16
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -112,6 +112,34 @@ def test_projection_host_validation_before_any_cuda_call(lib):
     assert g(*args(max_seqlen=0)) == pa.PA_ERR_MAX_SEQLEN
     assert g(*args(cu=None)) == pa.PA_ERR_NULL
     assert g(*args(batch=0, total=0)) == pa.PA_OK
+
+
+def test_fp8_host_validation_before_any_cuda_call(lib):
+    # keys per transposed-V row: 16*ceil(T/16) + 16*B
+    assert pa.pa_fp8_vt_keys(3, 100) == 112 + 48
+    assert pa.pa_fp8_vt_keys(1, 16) == 32 and pa.pa_fp8_vt_keys(0, 0) == 0
+    assert pa.pa_fp8_vt_keys(-1, 4) == -1
+    q = lib.pa_fp8_quantize_qkv
+    qargs = lambda **kw: (kw.get("q", 16), 16, 16, kw.get("cu", 16), kw.get("batch", 1), kw.get("total", 4), 1,
+                          kw.get("d", 128), 16, 16, kw.get("v8t", 16), kw.get("scales", 16), None)
+    assert q(*qargs(d=64)) == pa.PA_ERR_HEAD_DIM
+    assert q(*qargs(batch=0, total=3)) == pa.PA_ERR_SHAPE
+    assert q(*qargs(batch=0, total=0)) == pa.PA_OK
+    assert q(*qargs(q=None)) == pa.PA_ERR_NULL
+    assert q(*qargs(v8t=24)) == pa.PA_ERR_ALIGN
+    assert q(*qargs(scales=8)) == pa.PA_ERR_ALIGN
+    assert q(*qargs(total=128 * 65536)) == pa.PA_ERR_SHAPE
+    f = lib.pa_varlen_attn_fwd_fp8
+    fargs = lambda **kw: (16, 16, kw.get("v8t", 16), kw.get("scales", 16), 16, kw.get("batch", 1), kw.get("total", 4),
+                          1, kw.get("d", 128), kw.get("max_seqlen", 4), ctypes.c_float(kw.get("scale", 0.1)),
+                          kw.get("out", 16), 16, None)
+    assert f(*fargs(d=64)) == pa.PA_ERR_HEAD_DIM
+    assert f(*fargs(scale=math.nan)) == pa.PA_ERR_SCALE
+    assert f(*fargs(max_seqlen=0)) == pa.PA_ERR_MAX_SEQLEN
+    assert f(*fargs(scales=None)) == pa.PA_ERR_NULL
+    assert f(*fargs(scales=20)) == pa.PA_ERR_ALIGN
+    assert f(*fargs(out=8)) == pa.PA_ERR_ALIGN
+    assert f(*fargs(batch=3, total=0)) == pa.PA_OK
 
 
 def test_missing_library_fails_loudly(tmp_path):
