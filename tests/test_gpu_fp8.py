@@ -115,6 +115,9 @@ PACKS = {
     "ragged": ([1, 127, 128, 129, 300, 0, 513, 17], 3),
     "one_tile": ([128], 1),
     "odd_starts": ([5, 250, 3, 700, 9], 2),
+    "empty_ends": ([0, 0, 300, 0, 129, 0], 2),
+    # more segments than the scheduler stages in shared memory (4096)
+    "many_segments": ([int(n) for n in np.random.default_rng(5).integers(0, 40, 5000)], 1),
 }
 
 
