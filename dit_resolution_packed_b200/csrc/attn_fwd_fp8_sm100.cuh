@@ -610,9 +610,10 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
     const uint4* q, const uint4* k, const uint4* v, const int32_t* cu, int32_t batch, int32_t total, int32_t heads,
     const uint32_t* amax, uint2* q8, uint2* k8, uint8_t* v8t, int64_t vt_keys, float* scales) {
   constexpr int D = 128;
-  __shared__ uint8_t s_t[D][128 + 4];  // [channel][token] of this tile
+  __shared__ __align__(16) uint8_t s_t[D][128 + 4];  // [channel][token] of this tile (word-aligned rows)
   __shared__ float s_mv[D];
   __shared__ int64_t s_off[128];
+  __shared__ int s_vec[8];  // 16-token chunk goes out as one 16-byte store
   const int h = blockIdx.x;
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * 128;
   const float mq = fp8_mult(__ldg(amax)), mk = fp8_mult(__ldg(amax + 1));
@@ -643,37 +644,62 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
     scales[3] = 0.f;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < 128 * (D / 8); i += kQuantThreads) {
-    const int tt = i >> 4, c8 = i & 15;
-    const int64_t t = t0 + tt;
-    if (t >= total) continue;
-    const int64_t idx = (t * heads + h) * (D / 8) + c8;
-    q8[idx] = quant8(__ldg(q + idx), mq);
-    k8[idx] = quant8(__ldg(k + idx), mk);
-    const uint4 x = __ldg(v + idx);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  // q, k: 8 codes per 16-byte load; v: four tokens of one 8-channel chunk per thread, so
+  // that each channel's four codes go to the transposed tile as one 32-bit word
+  for (int i = threadIdx.x; i < 32 * (D / 8); i += kQuantThreads) {
+    const int tg = i >> 4, c8 = i & 15;
+    uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // [channel of the chunk]: 4 token bytes
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = c8 * 8 + 2 * e;
-      const float lo = __fmul_rn(__uint_as_float(w[e] << 16), s_mv[c]);
-      const float hi = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), s_mv[c + 1]);
-      const uint32_t pr = pack_e4m3x2_pair(f2_pack(lo, hi));
-      s_t[c][tt] = static_cast<uint8_t>(pr);
-      s_t[c + 1][tt] = static_cast<uint8_t>(pr >> 8);
+    for (int u = 0; u < 4; ++u) {
+      const int64_t t = t0 + tg * 4 + u;
+      if (t >= total) break;
+      const int64_t idx = (t * heads + h) * (D / 8) + c8;
+      q8[idx] = quant8(__ldg(q + idx), mq);
+      k8[idx] = quant8(__ldg(k + idx), mk);
+      const uint4 x = __ldg(v + idx);
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c8 * 8 + 2 * e;
+        const float lo = __fmul_rn(__uint_as_float(w[e] << 16), s_mv[c]);
+        const float hi = __fmul_rn(__uint_as_float(w[e] & 0xFFFF0000u), s_mv[c + 1]);
+        const uint32_t pr = pack_e4m3x2_pair(f2_pack(lo, hi));
+        pk[2 * e] |= (pr & 0xFFu) << (8 * u);
+        pk[2 * e + 1] |= ((pr >> 8) & 0xFFu) << (8 * u);
+      }
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) *reinterpret_cast<uint32_t*>(&s_t[c8 * 8 + e][tg * 4]) = pk[e];
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < D * 32; i += kQuantThreads) {
-    const int c = i >> 5, g = i & 31;
+  // v8^T rows, one warp per channel row: a 16-token chunk goes out as one 16-byte store
+  // when its tokens lie in one segment (equal key offsets: the offset grows at every
+  // segment start) and its first key is 16-byte aligned (decided once per block, the
+  // same for every row); the other tokens as bytes, four consecutive tokens per lane.
+  // Keys are in range for every valid cu_seqlens; the checks keep a malformed one (not
+  // validated here) from writing outside the buffer.
+  if (threadIdx.x < 8) {
+    const int tt0 = threadIdx.x * 16;
+    const int64_t t_first = t0 + tt0, key0 = t_first + s_off[tt0];
+    s_vec[threadIdx.x] = t_first + 15 < total && s_off[tt0] == s_off[tt0 + 15] && (key0 & 15) == 0 &&
+                         key0 >= 0 && key0 + 16 <= vt_keys;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int c = warp; c < D; c += kQuantThreads / 32) {
     uint8_t* row = v8t + static_cast<int64_t>(h * D + c) * vt_keys;
+    if (lane < 8 && s_vec[lane]) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(&s_t[c][lane * 16]);
+      *reinterpret_cast<uint4*>(row + t0 + lane * 16 + s_off[lane * 16]) = make_uint4(src[0], src[1], src[2], src[3]);
+    }
+    if (!s_vec[lane >> 2]) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tt = g * 4 + e;
-      const int64_t t = t0 + tt;
-      const int64_t key = t + s_off[tt];
-      // in range for every valid cu_seqlens; the check keeps a malformed one (not
-      // validated here) from writing outside the buffer
-      if (t < total && key >= 0 && key < vt_keys) row[key] = s_t[c][tt];
+      for (int e = 0; e < 4; ++e) {
+        const int tt = lane * 4 + e;
+        const int64_t t = t0 + tt;
+        const int64_t key = t + s_off[tt];
+        if (t < total && key >= 0 && key < vt_keys) row[key] = s_t[c][tt];
+      }
     }
   }
 }
