@@ -214,6 +214,69 @@ int prof_begin(cudaStream_t stream, cudaEvent_t* ev1) {
   return PA_OK;
 }
 
+// Schedule parameters of a forward call (the template maps are filled by the caller):
+// workspace slices, the pack, pair items (2^8 query rows), the status codes.
+pa::SchedParams forward_sched(const int32_t* cu, int32_t* status, uint8_t* ws, const WsLayout& L, int32_t batch,
+                              int32_t total, int32_t heads, int32_t max_seqlen, uint64_t row_bytes) {
+  pa::SchedParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  sp.cu = cu;
+  sp.status = status;
+  sp.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  sp.order = reinterpret_cast<int32_t*>(ws + L.order);
+  sp.item_start = reinterpret_cast<int32_t*>(ws + L.item_start);
+  sp.maps = ws + L.maps;
+  sp.row_bytes = row_bytes;
+  sp.batch = batch;
+  sp.total = total;
+  sp.heads = heads;
+  sp.max_seqlen = max_seqlen;
+  sp.rows_log2 = 8;
+  sp.err_cu = PA_ERR_CU_SEQLENS;
+  sp.err_max = PA_ERR_MAX_SEQLEN;
+  return sp;
+}
+
+// Attention-kernel parameters of a forward call, reading the schedule that `sp` describes.
+pa::FwdParams forward_params(const pa::SchedParams& sp, void* out, float* lse, float scale) {
+  pa::FwdParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.cu = sp.cu;
+  fp.out = out;
+  fp.lse = lse;
+  fp.counts = sp.counts;
+  fp.next_item = sp.counts + 2;
+  fp.order = sp.order;
+  fp.item_start = sp.item_start;
+  fp.maps = sp.maps;
+  fp.status = sp.status;
+  fp.heads = sp.heads;
+  fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
+  fp.err_timeout = PA_ERR_TIMEOUT;
+  return fp;
+}
+
+// Launches an attention kernel right behind the schedule kernel.  With `pdl`, as a
+// programmatic dependent launch: its prologue (barrier set-up, tensor-memory
+// allocation) overlaps the schedule kernel, whose results it reads only after
+// griddepcontrol.wait.
+template <class P>
+int launch_after_schedule(void (*kernel)(P), const P& params, int grid, size_t smem, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(pa::kFwdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, params) != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
 // Launches the projection GEMM (epilogue kEpi) on the persistent grid.
 template <int kEpi>
 int launch_gemm(const pa::GemmParams& gp, int dev, cudaStream_t stream) {
@@ -316,74 +379,27 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
   const WsLayout L = ws_layout(batch);
   if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
 
-  pa::SchedParams sp;
-  std::memset(&sp, 0, sizeof(sp));
+  pa::SchedParams sp = forward_sched(cu_seqlens, st->status, st->ws, L, batch, total_tokens, heads, max_seqlen,
+                                     static_cast<uint64_t>(heads) * head_dim * 2);
   const void* bases[3] = {q, k, v};
   for (int i = 0; i < 3; ++i) {
     if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
     sp.base[i] = bases[i];
   }
-  sp.cu = cu_seqlens;
-  sp.status = st->status;
-  sp.counts = reinterpret_cast<int32_t*>(st->ws + L.counts);
-  sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
-  sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
-  sp.maps = st->ws + L.maps;
-  sp.row_bytes = static_cast<uint64_t>(heads) * head_dim * 2;
-  sp.batch = batch;
-  sp.total = total_tokens;
-  sp.heads = heads;
-  sp.max_seqlen = max_seqlen;
-  sp.rows_log2 = 8;
-  sp.err_cu = PA_ERR_CU_SEQLENS;
-  sp.err_max = PA_ERR_MAX_SEQLEN;
   pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
 
-  pa::FwdParams fp;
-  fp.cu = cu_seqlens;
-  fp.out = out;
-  fp.lse = lse;
-  fp.counts = sp.counts;
-  fp.next_item = sp.counts + 2;
-  fp.order = sp.order;
-  fp.item_start = sp.item_start;
-  fp.maps = sp.maps;
-  fp.status = st->status;
-  fp.heads = heads;
-  fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
-  fp.err_timeout = PA_ERR_TIMEOUT;
+  const pa::FwdParams fp = forward_params(sp, out, lse, scale);
   const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
-
-  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
-  if (g_prof_on) {
-    if (g_prof_used == g_prof_events.size()) {
-      cudaEvent_t a, b;
-      if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return PA_ERR_CUDA;
-      g_prof_events.emplace_back(a, b);
-    }
-    ev0 = g_prof_events[g_prof_used].first;
-    ev1 = g_prof_events[g_prof_used].second;
-    ++g_prof_used;
-    cudaEventRecord(ev0, stream);
-  }
-  // Programmatic dependent launch: the attention kernel's prologue overlaps the
-  // schedule kernel, whose results it reads only after griddepcontrol.wait.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(pa::kFwdThreads);
-  cfg.dynamicSmemBytes = head_dim == 128 ? pa::FwdCfg<128>::kSmemBytes : pa::FwdCfg<64>::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = g_prof_on ? 0 : 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = head_dim == 128 ? cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<128>, fp)
-                                         : cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<64>, fp);
-  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (g_prof_on) cudaEventRecord(ev1, stream);
+  cudaEvent_t ev1 = nullptr;
+  if ((rc = prof_begin(stream, &ev1)) != PA_OK) return rc;
+  // (no programmatic overlap while profiling: the events then bracket the attention kernel alone)
+  rc = head_dim == 128 ? launch_after_schedule(pa::attn_fwd_kernel<128>, fp, grid, pa::FwdCfg<128>::kSmemBytes,
+                                               stream, !g_prof_on)
+                       : launch_after_schedule(pa::attn_fwd_kernel<64>, fp, grid, pa::FwdCfg<64>::kSmemBytes,
+                                               stream, !g_prof_on);
+  if (rc != PA_OK) return rc;
+  if (ev1) cudaEventRecord(ev1, stream);
   return PA_OK;
 }
 
@@ -762,58 +778,22 @@ int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, cons
   // (counts, work counter, order, item starts, tensor maps) before it is read.
   if (cudaMemsetAsync(st, 0, sizeof(int32_t), stream) != cudaSuccess) return PA_ERR_CUDA;
 
-  pa::SchedParams sp;
-  std::memset(&sp, 0, sizeof(sp));
+  pa::SchedParams sp = forward_sched(cu_seqlens, st, ws, L, batch, total_tokens, heads, max_seqlen,
+                                     static_cast<uint64_t>(heads) * head_dim * 2);
   const void* bases[3] = {q, k, v};
   for (int i = 0; i < 3; ++i) {
     if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
     sp.base[i] = bases[i];
   }
-  sp.cu = cu_seqlens;
-  sp.status = st;
-  sp.counts = reinterpret_cast<int32_t*>(ws + L.counts);
-  sp.order = reinterpret_cast<int32_t*>(ws + L.order);
-  sp.item_start = reinterpret_cast<int32_t*>(ws + L.item_start);
-  sp.maps = ws + L.maps;
-  sp.row_bytes = static_cast<uint64_t>(heads) * head_dim * 2;
-  sp.batch = batch;
-  sp.total = total_tokens;
-  sp.heads = heads;
-  sp.max_seqlen = max_seqlen;
-  sp.rows_log2 = 8;
-  sp.err_cu = PA_ERR_CU_SEQLENS;
-  sp.err_max = PA_ERR_MAX_SEQLEN;
   pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
 
-  pa::FwdParams fp;
-  fp.cu = cu_seqlens;
-  fp.out = out;
-  fp.lse = lse;
-  fp.counts = sp.counts;
-  fp.next_item = sp.counts + 2;
-  fp.order = sp.order;
-  fp.item_start = sp.item_start;
-  fp.maps = sp.maps;
-  fp.status = st;
-  fp.heads = heads;
-  fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
-  fp.err_timeout = PA_ERR_TIMEOUT;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound)));
-  cfg.blockDim = dim3(pa::kFwdThreads);
-  cfg.dynamicSmemBytes = head_dim == 128 ? pa::FwdCfg<128>::kSmemBytes : pa::FwdCfg<64>::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = head_dim == 128 ? cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<128>, fp)
-                                         : cudaLaunchKernelEx(&cfg, pa::attn_fwd_kernel<64>, fp);
-  if (le != cudaSuccess || cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  return PA_OK;
+  const pa::FwdParams fp = forward_params(sp, out, lse, scale);
+  const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
+  return head_dim == 128 ? launch_after_schedule(pa::attn_fwd_kernel<128>, fp, grid, pa::FwdCfg<128>::kSmemBytes,
+                                                 stream, true)
+                         : launch_after_schedule(pa::attn_fwd_kernel<64>, fp, grid, pa::FwdCfg<64>::kSmemBytes,
+                                                 stream, true);
 }
 
 int64_t pa_fp8_vt_keys(int32_t batch, int32_t total_tokens) {
@@ -905,64 +885,29 @@ int pa_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8t, cons
   const WsLayout L = ws_layout(batch);
   if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
 
-  pa::SchedParams sp;
-  std::memset(&sp, 0, sizeof(sp));
   const int64_t hd = static_cast<int64_t>(heads) * head_dim;
+  pa::SchedParams sp = forward_sched(cu_seqlens, st->status, st->ws, L, batch, total_tokens, heads, max_seqlen,
+                                     static_cast<uint64_t>(hd));
   if (!encode_u8(&sp.tmpl[0], q8, hd, total_tokens, hd) || !encode_u8(&sp.tmpl[1], k8, hd, total_tokens, hd) ||
       !encode_u8(&sp.tmpl[2], v8t, vt_keys, hd, vt_keys))
     return PA_ERR_CUDA;
   sp.base[0] = q8;
   sp.base[1] = k8;
   sp.base[2] = v8t;
-  sp.cu = cu_seqlens;
-  sp.status = st->status;
-  sp.counts = reinterpret_cast<int32_t*>(st->ws + L.counts);
-  sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
-  sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
-  sp.maps = st->ws + L.maps;
-  sp.row_bytes = static_cast<uint64_t>(hd);
-  sp.batch = batch;
-  sp.total = total_tokens;
-  sp.heads = heads;
-  sp.max_seqlen = max_seqlen;
-  sp.rows_log2 = 8;
   sp.v_keys_inner = 1;
-  sp.err_cu = PA_ERR_CU_SEQLENS;
-  sp.err_max = PA_ERR_MAX_SEQLEN;
   pa::schedule_kernel<<<1, pa::kSchedThreads, 0, stream>>>(sp);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
 
   pa::Fp8Params fp;
   std::memset(&fp, 0, sizeof(fp));
-  fp.f.cu = cu_seqlens;
-  fp.f.out = out;
-  fp.f.lse = lse;
-  fp.f.counts = sp.counts;
-  fp.f.next_item = sp.counts + 2;
-  fp.f.order = sp.order;
-  fp.f.item_start = sp.item_start;
-  fp.f.maps = sp.maps;
-  fp.f.status = st->status;
-  fp.f.heads = heads;
-  fp.f.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  fp.f.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
-  fp.f.err_timeout = PA_ERR_TIMEOUT;
+  fp.f = forward_params(sp, out, lse, scale);
   fp.scales = scales;
   const int grid = static_cast<int>(std::min<int64_t>(g_dev[dev].sms, item_bound));
   cudaEvent_t ev1 = nullptr;
   if ((rc = prof_begin(stream, &ev1)) != PA_OK) return rc;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(pa::kFwdThreads);
-  cfg.dynamicSmemBytes = pa::Fp8Cfg::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = g_prof_on ? 0 : 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, pa::attn_fwd_fp8_kernel, fp) != cudaSuccess || cudaGetLastError() != cudaSuccess)
-    return PA_ERR_CUDA;
+  if ((rc = launch_after_schedule(pa::attn_fwd_fp8_kernel, fp, grid, pa::Fp8Cfg::kSmemBytes, stream, !g_prof_on)) !=
+      PA_OK)
+    return rc;
   if (ev1) cudaEventRecord(ev1, stream);
   return PA_OK;
 }
