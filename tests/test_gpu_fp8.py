@@ -83,18 +83,18 @@ def _compare_full(p, out, lse, name, qz=None):
     T, H, _ = ref.shape
     tok = np.repeat(np.arange(T), H)
     head = np.tile(np.arange(H), T)
-    sig = parity.fp8_sigma(qh, kh, vh, cu, p["scale"], tok, head, ref.reshape(T * H, -1))
+    sig, bias = parity.fp8_sigma(qh, kh, vh, cu, p["scale"], tok, head, ref.reshape(T * H, -1))
     return parity.fp8_check(out.double().cpu().numpy().reshape(T * H, -1), lse.double().cpu().numpy().reshape(-1),
-                            ref.reshape(T * H, -1), rlse.reshape(-1), sig, name)
+                            ref.reshape(T * H, -1), rlse.reshape(-1), sig, bias, name)
 
 
 def _compare_rows(p, out, lse, tok, head, name, qz):
     qh, kh, vh = fp8.dequantized_qkv(qz)
     cu = p["cu_seqlens"].numpy()
     ref, rlse = oracle.varlen_attention(qh, kh, vh, cu, p["scale"], rows=(tok, head))
-    sig = parity.fp8_sigma(qh, kh, vh, cu, p["scale"], tok, head, ref)
+    sig, bias = parity.fp8_sigma(qh, kh, vh, cu, p["scale"], tok, head, ref)
     go, gl = parity.gather_rows(out, lse, tok, head)
-    return parity.fp8_check(go, gl, ref, rlse, sig, name)
+    return parity.fp8_check(go, gl, ref, rlse, sig, bias, name)
 
 
 def _check_quantiser(pa, p, qz_dev, rows=None, qz=None):
