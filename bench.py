@@ -9,6 +9,13 @@ attention kernel) on inputs resident in HBM; L2 is flushed between timed steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
 
+Beside the headline the line carries: ``steady_state`` (at least --steady-s seconds of
+back-to-back calls, with the clock samples of that region and the roofline against the
+sustained bf16 figure), ``per_config`` (the other workloads, each with its kernel's
+roofline), ``short_segments`` (packs of small images, where the path is bound by HBM:
+unique bytes / time against the measured copy bandwidth), and the backward, the
+projections and the FP8 variant of the same pack.
+
 With N > 1 (torchrun, one rank per GPU) every rank runs its own pack of the same
 shape (independent replicas: the forward has no exchange step), the timed
 region is bracketed by barriers, and the time is the max over ranks.
@@ -111,17 +118,11 @@ class ClockSampler:
                 continue
             self.rows.append([ts] + parts[1:])
 
-    def stop(self, t0, t1):
-        """Summary of the samples taken in [t0, t1] (host wall-clock seconds)."""
+    def summary(self, t0, t1):
+        """Summary of the samples taken in [t0, t1] (host wall-clock seconds); the sampler keeps running."""
         if self.proc is None:
             return None
-        time.sleep(2.5 * self.PERIOD_MS / 1e3)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = [r for r in self.rows if t0 <= r[0] <= t1]
+        rows = [r for r in list(self.rows) if t0 <= r[0] <= t1]
         in_region = bool(rows)
         if not rows and self.rows:  # region shorter than the sampling period: nearest sample (within 1 s)
             near = min(self.rows, key=lambda r: abs(r[0] - t0))
@@ -139,6 +140,18 @@ class ClockSampler:
                 "power_w_median": statistics.median(pw) if pw else None,
                 "window": "samples taken inside the timed region" if in_region
                           else "timed region shorter than the sampling period: nearest sample"}
+
+    def stop(self, t0=None, t1=None):
+        """Stops sampling; returns the summary of [t0, t1] when a window is given."""
+        if self.proc is None:
+            return None
+        time.sleep(2.5 * self.PERIOD_MS / 1e3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        return self.summary(t0, t1) if t0 is not None else None
 
 
 def workload_desc(cfg):
@@ -222,6 +235,109 @@ def traffic_for_current_kernel():
     return rec
 
 
+def time_steps(call, flush, stream, warmup, steps, world, device, flush_each=True):
+    """W untimed calls, then K calls each bracketed by CUDA events on the launching stream (L2
+    flushed before every call when flush_each), barriers + synchronize around the region.
+    Returns (per-call ms list, host t0, host t1) with the per-call times max-reduced over ranks."""
+    for _ in range(warmup):
+        if flush_each:
+            flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for a, b in ev:
+        if flush_each:
+            flush.fill_(1.0)  # evict the operands from L2 (untimed)
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t1 = time.time()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor(ms, dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.tolist()
+    return ms, t0, t1
+
+
+def kernel_ms(pa, call, flush, steps, flush_each=True):
+    """Average duration (ms) of the library's main kernel over `steps` calls, from the events
+    the library records around it on its launch stream; also the host seconds the run took."""
+    pa.pa_profile_read()  # clear
+    pa.pa_profile_enable(True)
+    t0 = time.time()
+    for _ in range(steps):
+        if flush_each:
+            flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    dt = time.time() - t0
+    pa.pa_profile_enable(False)
+    tot, n = pa.pa_profile_read()
+    return tot / max(1, n), dt
+
+
+def unique_bytes(T, H, d):
+    """Algorithmic HBM bytes of one forward call: q, k, v read and out written (bf16), lse written (fp32)."""
+    return 4.0 * T * H * d * 2 + 4.0 * T * H
+
+
+class Pack:
+    """Device-resident inputs and outputs of one workload, and the C-ABI call on them."""
+
+    def __init__(self, pa, cfg, device, stream, seed_offset=0):
+        self.pa, self.cfg, self.stream = pa, cfg, stream
+        p = workloads.make_inputs(dict(cfg, seed=int(cfg["seed"]) + seed_offset))
+        self.p = p
+        self.segs = [int(n) for n in cfg["segments"]]
+        self.T, self.H, self.d = sum(self.segs), int(cfg["heads"]), int(cfg["head_dim"])
+        self.flops = workloads.valid_flops(self.segs, self.H, self.d)
+        self.bytes = unique_bytes(self.T, self.H, self.d)
+        self.q, self.k, self.v = (p[n].to(device) for n in ("q", "k", "v"))
+        self.cu = p["cu_seqlens"].to(device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.T, self.H, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        pa = self.pa
+        rc = pa.pa_varlen_attn_fwd(self.q, self.k, self.v, self.cu, self.p["max_seqlen"], self.p["scale"],
+                                   self.out, self.lse, self.stream)
+        if rc != pa.PA_OK:
+            raise pa.PackAttnError(rc, "pa_varlen_attn_fwd")
+
+
+def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5):
+    """Per-call time of one pack (L2 flushed before every call) and its kernel alone; the step
+    count is the bench's, capped so that the region stays under about `target_s` seconds."""
+    pack()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    pack()
+    torch.cuda.synchronize()
+    est = max(time.time() - t0, 1e-5)
+    steps = max(5, min(args.steps, int(target_s / est)))
+    ms, _, _ = time_steps(pack, flush, stream, args.warmup, steps, world, device)
+    kms, _ = kernel_ms(pa, pack, flush, steps)
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, pack.cfg["name"])
+    call_ms = sum(ms) / len(ms)
+    return dict(steps=steps, ms_per_call=call_ms, kernel_ms=kms,
+                tflops=pack.flops * world / (call_ms * 1e-3) / 1e12,
+                kernel_tflops=pack.flops / (kms * 1e-3) / 1e12,
+                gbs=pack.bytes * world / (call_ms * 1e-3) / 1e9,
+                kernel_gbs=pack.bytes / (kms * 1e-3) / 1e9)
+
+
+def head_kernel_name(d):
+    return "attn_fwd_kernel<128>" if d == 128 else "attn_fwd_kernel<64>"
+
+
 def run_ours(args, world, rank, local):
     import dit_resolution_packed_b200 as pa
     if not torch.cuda.is_available():
@@ -229,71 +345,46 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     cfg = workloads.load_config(args.config)
-    cfg_r = dict(cfg, seed=int(cfg["seed"]) + 7919 * rank)  # each replica its own data, same shapes
-    p = workloads.make_inputs(cfg_r)
-    segs = cfg["segments"]
-    T, H, d = sum(segs), cfg["heads"], cfg["head_dim"]
-    flops = workloads.valid_flops(segs, H, d)
-    q, k, v = (p[n].to(device) for n in ("q", "k", "v"))
-    cu = p["cu_seqlens"].to(device)
-    out = torch.empty_like(q)
-    lse = torch.empty(T, H, dtype=torch.float32, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
+    head = Pack(pa, cfg, device, stream, seed_offset=7919 * rank)  # each replica its own data, same shapes
+    p, segs, T, H, d, flops = head.p, head.segs, head.T, head.H, head.d, head.flops
+    q, k, v, cu, out, lse = head.q, head.k, head.v, head.cu, head.out, head.lse
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    call = head
 
-    def call():
-        rc = pa.pa_varlen_attn_fwd(q, k, v, cu, p["max_seqlen"], p["scale"], out, lse, stream)
-        if rc != pa.PA_OK:
-            raise pa.PackAttnError(rc, "pa_varlen_attn_fwd")
-
-    # the clock sampler runs from here on (nvidia-smi needs a moment to start)
+    # the clock sampler runs from here to the end; each record keeps the samples of its own region
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        call()
-    torch.cuda.synchronize()
+        time.sleep(0.3)  # nvidia-smi needs a moment to start
+
+    # ---- headline: K calls after W warm-up calls, L2 flushed before each (a burst of K calls)
+    step_ms, t_region0, t_region1 = time_steps(call, flush, stream, args.warmup, args.steps, world, device)
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
-        raise pa.PackAttnError(rc, "warm-up")
-
-    # ---- device-resident timed region: it follows the warm-up directly (no idle gap that
-    # would let the GPU cool below its power limit), and the clock samples kept are the
-    # ones taken inside it
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    t_region0 = time.time()
-    for i in range(args.steps):
-        flush.fill_(1.0)  # evict q/k/v/out from L2 between steps (untimed)
-        ev[i][0].record(stream)
-        call()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    t_region1 = time.time()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    # attention kernel alone (for the roofline): the library brackets it with
-    # events on its launch stream; the schedule kernel is outside the events
-    pa.pa_profile_read()  # clear
-    pa.pa_profile_enable(True)
-    t_prof0 = time.time()
-    for i in range(args.steps):
-        flush.fill_(1.0)
-        call()
-    torch.cuda.synchronize()
-    t_prof = time.time() - t_prof0
-    pa.pa_profile_enable(False)
-    clock_rec = clocks.stop(t_region0, t_region1) if clocks else None
-    kern_ms_total, kern_n = pa.pa_profile_read()
+        raise pa.PackAttnError(rc, "timed region")
+    # attention kernel alone (for the roofline): the library brackets it with events on its
+    # launch stream; the schedule kernel is outside the events
+    kern_avg_ms, t_prof = kernel_ms(pa, call, flush, args.steps)
+    clock_rec = clocks.summary(t_region0, t_region1) if clocks else None
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, "timed region")
     q10, q50, q90 = (float(x) for x in np.percentile(step_ms, [10, 50, 90]))
-    total_ms = allreduce_max(sum(step_ms), world, device)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = sum(step_ms) / args.steps
     value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---- steady state under the board's power limit: back-to-back calls of the same pack for
+    # at least `steady_s` seconds (no flush between calls: the 158 MB of operands exceed the
+    # 126 MB L2), per-call events and the kernel's own events, clock samples inside the region
+    n_ss = max(args.steps, int(args.steady_s / max(ms_per_step * 1e-3, 1e-6)) + 1)
+    ss_ms, ss_t0, ss_t1 = time_steps(call, flush, stream, 0, n_ss, world, device, flush_each=False)
+    ss_kern_ms, _ = kernel_ms(pa, call, flush, n_ss, flush_each=False)
+    ss_clock = clocks.summary(ss_t0, ss_t1 + 0.02) if clocks else None
+    rc = pa.pa_get_error(stream)
+    if rc != pa.PA_OK:
+        raise pa.PackAttnError(rc, "steady-state region")
+    ss_call_ms = sum(ss_ms) / len(ss_ms)
 
     # ---- backward (the gradients of the same call): out and lse from the forward above, dout a
     # seeded N(0,1) tensor; same warm-up, step count and L2 flush as the forward
@@ -409,7 +500,10 @@ def run_ours(args, world, rank, local):
             raise pa.PackAttnError(rc, "fp8 region")
         fp8_rec = dict(quant_ms=quant_ms, fp8_ms=fp8_ms, both_ms=both_ms, t_prof=t_fprof,
                        kern_s=fkern_ms_total / max(1, fkern_n) * 1e-3,
-                       quant_bytes=15.0 * T * H * d)  # amax pass reads 6 B, quantise pass reads 6 B + writes 3 B
+                       # algorithmic bytes: q, k, v read once (6 B per element) and the E4M3 codes
+                       # written (3 B); the two-pass quantiser moves 15 B (the amax pass reads
+                       # q, k, v once more)
+                       quant_bytes=9.0 * T * H * d, quant_bytes_moved=15.0 * T * H * d)
 
     # ---- end to end through the public API with host buffers (pinned): every step copies its
     # q, k, v, cu_seqlens host -> device and its out, lse device -> host inside the timed region.
@@ -468,29 +562,84 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
     d2h = hout[0].numel() * hout[0].element_size() + hlse[0].numel() * hlse[0].element_size()
 
+    # ---- every other configuration of the workload list, and the short-segment regime: the same
+    # call, L2 flushed before each call, step count capped per pack
+    per_config = {}
+    if not args.no_configs:
+        del bufs, hq, hk, hv, hout, hlse
+        for name in workloads.CONFIG_NAMES + workloads.SHORT_PACK_NAMES:
+            if name == args.config:
+                continue
+            pk = Pack(pa, workloads.load_config(name), device, stream, seed_offset=7919 * rank)
+            rec = measure_pack(pa, pk, flush, stream, args, world, device)
+            rec.update(tokens=pk.T, segments=len(pk.segs), heads=pk.H, head_dim=pk.d, valid_flops=pk.flops,
+                       unique_bytes=pk.bytes)
+            per_config[name] = rec
+            del pk
+            torch.cuda.empty_cache()
+    if clocks:
+        clocks.stop()
+
     if rank != 0:
         return 0
     peaks, peak_src = load_peaks()
-    kern_avg_s = kern_ms_total / max(1, kern_n) * 1e-3
+    kern_avg_s = kern_avg_ms * 1e-3
     achieved = flops / kern_avg_s / 1e12
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     # The roofline's kernel is timed inside a run of back-to-back steps; once that run is
     # long enough to settle under the board's power limit (>= 0.25 s), its denominator is
     # the sustained cuBLAS figure, else the burst one.
     sustained = t_prof >= 0.25
-    bpeak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])) \
-        if t_bprof >= 0.25 else peak_burst
+    peak = peak_sust if sustained else peak_burst
+    bpeak = peak_sust if t_bprof >= 0.25 else peak_burst
     bpeak_src = (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_bprof:.2f} s of back-to-back steps)"
                  if t_bprof >= 0.25 else f"bf16_tflops ({peak_src}, burst)")
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])) if sustained \
-        else peak_burst
     trec = traffic_for_current_kernel()
+    ss_achieved = flops / (ss_kern_ms * 1e-3) / 1e12
+    steady = {
+        "what": (f"{n_ss} back-to-back calls of the same pack, no idle gap and no L2 flush between them "
+                 f"(q, k, v, out: {head.bytes / 1e6:.0f} MB > 126 MB L2); per-call CUDA events"),
+        "region_s": ss_t1 - ss_t0, "calls": n_ss, "ms_per_call": ss_call_ms,
+        "value": flops * world / (ss_call_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "pct_of_bf16_sustained": 100.0 * flops / (ss_call_ms * 1e-3) / 1e12 / peak_sust,
+        "roofline": {"bound": "tensor", "kernel": head_kernel_name(d), "achieved": ss_achieved,
+                     "peak": peak_sust, "unit": "TFLOP/s", "frac": ss_achieved / peak_sust,
+                     "peak_source": f"bf16_tflops_sustained ({peak_src}; cuBLAS timed back to back under the "
+                                    "power limit)",
+                     "frac_of_burst": ss_achieved / peak_burst},
+        "clocks": ss_clock,
+    }
+    if ss_clock and ss_clock.get("sm_mhz"):
+        # clock-normalised rate: valid FLOPs per SM clock cycle of the whole GPU
+        steady["flops_per_sm_cycle"] = flops / (ss_kern_ms * 1e-3) / (ss_clock["sm_mhz"] * 1e6)
+    configs_rec, short_rec = {}, {}
+    for name, rec in per_config.items():
+        r = {"tokens": rec["tokens"], "segments": rec["segments"], "heads": rec["heads"],
+             "head_dim": rec["head_dim"], "steps": rec["steps"], "ms_per_call": rec["ms_per_call"],
+             "value": rec["tflops"], "unit": "TFLOP/s", "pct_of_bf16_peak": 100.0 * rec["tflops"] / world / peak_burst,
+             "kernel": {"name": head_kernel_name(rec["head_dim"]), "ms": rec["kernel_ms"],
+                        "achieved": rec["kernel_tflops"], "frac": rec["kernel_tflops"] / peak_burst,
+                        "peak": peak_burst, "peak_source": f"bf16_tflops ({peak_src}, burst)"}}
+        if name in workloads.SHORT_PACK_NAMES or name == "tiny":
+            # short-segment regime: bound by HBM (per-segment intensity about L/2 FLOP per byte, below
+            # the ridge of about 259 FLOP/B for L < ~520); unique bytes / time
+            r["hbm"] = {"bound": "hbm", "unique_bytes": rec["unique_bytes"], "achieved": rec["gbs"],
+                        "kernel_achieved": rec["kernel_gbs"], "peak": hbm, "unit": "GB/s",
+                        "frac": rec["gbs"] / world / hbm, "kernel_frac": rec["kernel_gbs"] / hbm,
+                        "peak_source": f"hbm_gbs ({peak_src}, copy bandwidth)"}
+            short_rec[name] = r
+        else:
+            configs_rec[name] = r
     line = {
         "metric": BASELINE_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_desc(cfg), l2="flushed between timed steps (256 MiB write, untimed)",
-                       gpu_state="timed region follows the warm-up with no idle gap (power-limited steady state)",
+                       gpu_state=(f"{args.steps} calls right after {args.warmup} warm-up calls, L2 flushed "
+                                  f"before each: a burst of about {sum(step_ms):.1f} ms of GPU time; the "
+                                  "power-limited steady state is the `steady_state` record"),
                        parallelism=f"{world} independent replica(s), no collective"),
         "pct_of_bf16_peak": 100.0 * value / world / peak_burst,
         "pct_of_bf16_sustained": 100.0 * value / world / float(
@@ -502,7 +651,7 @@ def run_ours(args, world, rank, local):
                      "peak_source": (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_prof:.2f} s "
                                      "of back-to-back steps)") if sustained
                                     else f"bf16_tflops ({peak_src}, burst; kernel timed over {t_prof:.3f} s)",
-                     "kernel": "attn_fwd_kernel<128>" if d == 128 else "attn_fwd_kernel<64>",
+                     "kernel": head_kernel_name(d),
                      "traffic": (trec or {}).get("dram_bytes_per_launch"),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
@@ -535,6 +684,9 @@ def run_ours(args, world, rank, local):
                           "ms_per_step": fp8_rec["fp8_ms"], "launches_per_step": 2},
             "quantiser": {"ms_per_step": fp8_rec["quant_ms"], "launches_per_step": 3,
                           "roofline": {"bound": "hbm", "unit": "GB/s", "bytes_per_call": fp8_rec["quant_bytes"],
+                                       "bytes_note": "algorithmic: q, k, v read once + E4M3 codes written "
+                                                     "(9 B per element); the two-pass kernels move "
+                                                     "%.0f B per call" % fp8_rec["quant_bytes_moved"],
                                        "achieved": fp8_rec["quant_bytes"] / (fp8_rec["quant_ms"] * 1e-3) / 1e9,
                                        "peak": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
                                        "frac": fp8_rec["quant_bytes"] / (fp8_rec["quant_ms"] * 1e-3) / 1e9 /
@@ -558,6 +710,9 @@ def run_ours(args, world, rank, local):
         },
         "gpu_launches": 2 * args.steps,  # schedule + attention kernel per step, headline timed region
         "clocks": clock_rec,
+        "steady_state": steady,
+        "per_config": configs_rec or None,
+        "short_segments": short_rec or None,
     }
     if world == 1 and not args.no_cpu_baseline:
         r, rows, secs, threads = oracle_sample_rate(p, cfg, args.cpu_seconds)
@@ -635,9 +790,12 @@ def main():
     ap.add_argument("--steps", type=int, default=1500)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--config", default="mixed", choices=workloads.CONFIG_NAMES)
+    ap.add_argument("--config", default="mixed", choices=workloads.CONFIG_NAMES + workloads.SHORT_PACK_NAMES)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration and short-segment records")
+    ap.add_argument("--steady-s", type=float, default=0.6,
+                    help="seconds of back-to-back calls in the steady-state record")
     ap.add_argument("--packing-study", action="store_true",
                     help="padded vs bucketed vs packed layouts of the training image mix (one GPU)")
     args = ap.parse_args()

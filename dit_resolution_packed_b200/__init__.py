@@ -78,6 +78,10 @@ def load_library(path=None):
     lib.pa_version.argtypes = []
     lib.pa_release_workspace.restype = None
     lib.pa_release_workspace.argtypes = []
+    lib.pa_set_short_packing.restype = None
+    lib.pa_set_short_packing.argtypes = [ctypes.c_int]
+    lib.pa_schedule_stats.restype = ctypes.c_int
+    lib.pa_schedule_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
     lib.pa_set_wait_limit_ms.restype = None
     lib.pa_set_wait_limit_ms.argtypes = [ctypes.c_int]
     lib.pa_selftest_wait_timeout.restype = ctypes.c_int
@@ -359,6 +363,24 @@ def pa_version():
 
 def pa_release_workspace():
     load_library().pa_release_workspace()
+
+
+def pa_set_short_packing(on):
+    """C ``pa_set_short_packing``: consecutive short segments share 128-row tiles (default on)."""
+    load_library().pa_set_short_packing(1 if on else 0)
+
+
+def pa_schedule_stats(stream=None):
+    """C ``pa_schedule_stats``: the tile ledger of the last forward call on ``stream`` as a dict
+    (items, units, score_tiles, useful_pairs, groups, grouped_segments, tile_utilisation)."""
+    out = (ctypes.c_int64 * 6)()
+    rc = load_library().pa_schedule_stats(_stream_handle(stream), out)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_schedule_stats")
+    keys = ("items", "units", "score_tiles", "useful_pairs", "groups", "grouped_segments")
+    rec = dict(zip(keys, (int(x) for x in out)))
+    rec["tile_utilisation"] = rec["useful_pairs"] / (rec["score_tiles"] * 16384.0) if rec["score_tiles"] else 0.0
+    return rec
 
 
 def pa_set_wait_limit_ms(ms):

@@ -300,7 +300,7 @@ template <bool kPartial, bool kNeg>
 __device__ __forceinline__ void softmax_tile_fp8(const uint64_t (&v)[64], int kv_valid, bool first, float c,
                                                  uint32_t tO, uint32_t p_row, uint32_t sw, float& m, float& l,
                                                  float& lr, uint64_t* p_full_half, int lane) {
-  const float xmax = row_extreme<kPartial, kNeg>(v, kv_valid) * c;
+  const float xmax = row_extreme<kPartial, kNeg>(v, 0, kv_valid) * c;
   bool rescale = false;
   float alpha = 1.f;
   if (first) {

@@ -12,7 +12,9 @@
 // than kRescaleLog2 (then O and l are rescaled); otherwise P <= 2^kRescaleLog2
 // and the result is unchanged, because out and lse do not depend on m.
 //
-// Work item = (segment, head, pair of 128-row query tiles).  Items are taken
+// Work item = (unit, head, pair of 128-row query tiles), a unit being a segment
+// alone or a group of consecutive short segments that share tiles (the scheduler
+// forms them; each row then sees only its own segment's keys).  Items are taken
 // longest first from a global counter by the producer warp (dynamic
 // longest-processing-time scheduling) and handed to the other warps through a
 // two-slot shared-memory ring.  CTA layout, 12 warps:
@@ -40,12 +42,26 @@ namespace pa {
 // stay far from fp32 overflow.  Measured on B200: 12 instead of 8 saves ~2 % on a
 // single 16384-token segment (fewer O rescales), nothing elsewhere.
 constexpr float kRescaleLog2 = 12.0f;
-// In every group of four key pairs of a full score tile at head_dim 128, this many
-// are exponentiated on the FMA pipe (polynomial, max relative error below 1e-4,
-// far under the bf16 rounding of P) instead of the MUFU unit.  Measured on B200
-// with the warp-wide MMA issuer: 1 of 4 gains ~2 % at d = 128; at d = 64 it loses
-// ~1 %, and 2 of 4 spills registers.
-constexpr int kPolyPairsPer4 = 1;
+// In every group of four key pairs of a full score tile, this many are
+// exponentiated on the FMA pipe (polynomial, max relative error below 1e-4, far
+// under the bf16 rounding of P) instead of the MUFU unit, per head_dim.  Measured
+// on B200 with the warp-wide MMA issuer: 1 of 4 gains ~2 % at d = 128.
+#ifndef PA_POLY_PAIRS_D128
+#define PA_POLY_PAIRS_D128 1
+#endif
+#ifndef PA_POLY_PAIRS_D64
+#define PA_POLY_PAIRS_D64 0
+#endif
+template <int D>
+constexpr int kPolyPairsPer4 = D == 128 ? PA_POLY_PAIRS_D128 : PA_POLY_PAIRS_D64;
+// Normaliser of the output at head_dim 128: 1 = the sum of the bf16-rounded weights
+// that P.V uses (each output row an exact convex combination of value rows; three
+// more instructions per key pair), 0 = the fp32 sum of the unrounded weights.
+#ifndef PA_NORM_ROUNDED_D128
+#define PA_NORM_ROUNDED_D128 1
+#endif
+static_assert(PA_POLY_PAIRS_D128 >= 0 && PA_POLY_PAIRS_D128 <= 4 && PA_POLY_PAIRS_D64 >= 0 && PA_POLY_PAIRS_D64 <= 4,
+              "polynomial share out of range");
 constexpr int kFwdThreads = 384;
 // Register split of the 384-thread block launched at 168 registers per thread
 // (384 x 168 = 64512): the two softmax warpgroups rise to 216, the producer /
@@ -92,8 +108,10 @@ struct FwdParams {
   const int32_t* order;
   const int32_t* item_start;
   const uint8_t* maps;        // [B][3] tensor maps: q, k, v
+  const int32_t* info;        // [B] unit descriptors (short-segment groups); nullptr: one unit per segment
   int32_t* status;
   int32_t heads;
+  int32_t batch;
   float scale_log2;           // scale * log2(e)
   uint64_t wait_limit_ns;
   int32_t err_timeout;
@@ -106,15 +124,22 @@ struct Bars {
   uint64_t p_full[2][2];  // [tile][half]: P columns of keys 0-63 / 64-127 are in tensor memory
   uint64_t sched_full[2], sched_empty[2];  // work-item hand-off from the producer
   uint64_t drain;
-  int32_t sched_item[2][8];  // decoded items: seg, beg, len, head, q0, nkv, two, id; seg < 0 = done
+  int32_t sched_item[2][10];  // decoded items (WorkItem fields in order); seg < 0 = done
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// A work item: query tiles 0 and 1 of one unit and head.  For a segment alone,
+// tile t holds rows [q0 + 128 t, q0 + 128 t + 128) of the segment and meets all
+// nkv key tiles.  For a group of short segments (n0 > 0), tile 0 holds the unit's
+// tokens [0, n0) and tile 1 the tokens [n0, len); tile t meets only key tile t,
+// which starts at the same token as its query tile.
 struct WorkItem {
   int32_t seg, beg, len, head, q0, nkv;
   bool two;    // second query tile has rows
   int32_t id;  // index in the longest-first order
+  int32_t n0;  // group split (tokens of tile 0); 0: a segment alone
+  int32_t kt;  // score tiles per query tile: nkv alone, 1 in a group
 };
 
 __device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p, int32_t n_sorted) {
@@ -127,13 +152,26 @@ __device__ __forceinline__ WorkItem decode_item(int32_t item, const FwdParams& p
   w.seg = __ldg(p.order + lo);
   const int32_t local = item - __ldg(p.item_start + lo);
   w.beg = __ldg(p.cu + w.seg);
+  w.id = item;
+  const int32_t inf = p.info != nullptr ? __ldg(p.info + w.seg) : -1;
+  if (inf >= 0) {  // a group of short segments: one item per head
+    w.n0 = inf & 0x1ff;
+    w.len = (inf >> 9) & 0x1ff;
+    w.head = local;
+    w.q0 = 0;
+    w.two = w.len > w.n0;
+    w.nkv = w.two ? 2 : 1;
+    w.kt = 1;
+    return w;
+  }
   w.len = __ldg(p.cu + w.seg + 1) - w.beg;
   const int32_t npairs = (w.len + 255) >> 8;
   w.head = local / npairs;
   w.q0 = (local - w.head * npairs) * 256;
   w.nkv = (w.len + 127) >> 7;
   w.two = w.q0 + 128 < w.len;
-  w.id = item;
+  w.n0 = 0;
+  w.kt = w.nkv;
   return w;
 }
 
@@ -148,6 +186,8 @@ __device__ __forceinline__ void store_item(volatile int32_t* d, const WorkItem& 
   d[5] = w.nkv;
   d[6] = w.two ? 1 : 0;
   d[7] = w.id;
+  d[8] = w.n0;
+  d[9] = w.kt;
 }
 __device__ __forceinline__ WorkItem load_item(const volatile int32_t* d) {
   WorkItem w;
@@ -159,6 +199,8 @@ __device__ __forceinline__ WorkItem load_item(const volatile int32_t* d) {
   w.nkv = d[5];
   w.two = d[6] != 0;
   w.id = d[7];
+  w.n0 = d[8];
+  w.kt = d[9];
   return w;
 }
 
@@ -213,6 +255,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
     fence_tmap_acquire(mk);
     fence_tmap_acquire(mv);
     const int32_t xcol = w.head * D;
+    const int32_t step = w.n0 ? w.n0 : 128;  // first token of query / key tile 1 within the unit
     if (!(ok = mbar_wait(&bars->q_empty, (q_round & 1u) ^ 1u, wc))) break;
     mbar_arrive_expect_tx(&bars->q_full, (w.two ? 2u : 1u) * C::kTileBytes);
     q_armed = true;
@@ -221,7 +264,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
     for (int cb = 0; cb < C::kColBlocks; ++cb) {
       tma_load_2d(smem + C::kOffQ + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0, &bars->q_full);
       if (w.two)
-        tma_load_2d(smem + C::kOffQ + C::kTileBytes + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0 + 128,
+        tma_load_2d(smem + C::kOffQ + C::kTileBytes + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0 + step,
                     &bars->q_full);
     }
     ++q_round;
@@ -236,7 +279,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
         const void* m = which ? mv : mk;
 #pragma unroll
         for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, j * 128, &bars->kv_full[slot]);
+          tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, j * step, &bars->kv_full[slot]);
         if (++slot == C::kSlots) {
           slot = 0;
           phase ^= 1u;
@@ -324,6 +367,60 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
     if (got <= 0) break;
     if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
     ++q_round;
+    if (w.n0) {
+      // A group of short segments: S_t = Q_t K_t^T and O_t = P_t V_t, tile t meeting only
+      // key tile t.  The ring holds K_0, V_0 [, K_1, V_1] in this order.
+      const int ntile = w.two ? 2 : 1;
+      int rs[4];
+      uint32_t rp[4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        int s2 = slot + o;
+        uint32_t ph2 = phase;
+        if (s2 >= C::kSlots) {
+          s2 -= C::kSlots;
+          ph2 ^= 1u;
+        }
+        rs[o] = s2;
+        rp[o] = ph2;
+      }
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t == ntile) break;
+        if (!(ok = mbar_wait(&bars->kv_full[rs[2 * t]], rp[2 * t], wc))) break;
+        tc_fence_after();
+        issue_s<D>(leader, tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + rs[2 * t] * C::kTileBytes);
+        mma_commit_if(leader, &bars->s_full[t]);
+        mma_commit_if(leader, &bars->kv_empty[rs[2 * t]]);
+      }
+      if (!ok) break;
+      mma_commit_if(leader, &bars->q_empty);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t == ntile) break;
+        if (!(ok = mbar_wait(&bars->o_empty[t], ((oe_ph >> t) & 1u) ^ 1u, wc))) break;
+        oe_ph ^= 1u << t;
+        const int vs = rs[2 * t + 1];
+        if (!(ok = mbar_wait(&bars->kv_full[vs], rp[2 * t + 1], wc))) break;
+        if (!(ok = mbar_wait(&bars->p_full[t][0], (p_ph >> t) & 1u, wc))) break;
+        tc_fence_after();
+        issue_pv_half<D>(leader, tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 0, false);
+        if (!(ok = mbar_wait(&bars->p_full[t][1], (p_ph >> t) & 1u, wc))) break;
+        p_ph ^= 1u << t;
+        tc_fence_after();
+        issue_pv_half<D>(leader, tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 1, true);
+        mma_commit_if(leader, &bars->o_full[t]);
+        mma_commit_if(leader, &bars->kv_empty[vs]);
+      }
+      if (!ok) break;
+      slot = w.two ? rs[3] + 1 : rs[1] + 1;
+      phase = w.two ? rp[3] : rp[1];
+      if (slot == C::kSlots) {
+        slot = 0;
+        phase ^= 1u;
+      }
+      continue;
+    }
     int ks = slot;
     if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
     if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
@@ -384,11 +481,11 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
 
 // ------------------------------------------------------------------ softmax + epilogue
 // Row extreme of the 128 scores (64 register pairs): max (kNeg = false) or min
-// (kNeg = true, for a negative scale), keys >= kv_valid excluded when kPartial.
+// (kNeg = true, for a negative scale), only keys in [kv_lo, kv_hi) when kPartial.
 // Eight independent chains of three-input max/min keep the dependency depth
 // near 10.
 template <bool kPartial, bool kNeg>
-__device__ __forceinline__ float row_extreme(const uint64_t (&v)[64], int kv_valid) {
+__device__ __forceinline__ float row_extreme(const uint64_t (&v)[64], int kv_lo, int kv_hi) {
   const float fill = kNeg ? INFINITY : -INFINITY;
   float a[8];
 #pragma unroll
@@ -399,8 +496,8 @@ __device__ __forceinline__ float row_extreme(const uint64_t (&v)[64], int kv_val
     for (int i = 0; i < 8; ++i) {
       float x0 = f2_lo(v[k + i]), x1 = f2_hi(v[k + i]);
       if (kPartial) {
-        x0 = (2 * (k + i) < kv_valid) ? x0 : fill;
-        x1 = (2 * (k + i) + 1 < kv_valid) ? x1 : fill;
+        x0 = (2 * (k + i) >= kv_lo && 2 * (k + i) < kv_hi) ? x0 : fill;
+        x1 = (2 * (k + i) + 1 >= kv_lo && 2 * (k + i) + 1 < kv_hi) ? x1 : fill;
       }
       a[i] = kNeg ? min3f(a[i], x0, x1) : max3f(a[i], x0, x1);
     }
@@ -414,11 +511,13 @@ __device__ __forceinline__ float row_extreme(const uint64_t (&v)[64], int kv_val
 // tensor memory in two halves of 64 keys; each half is handed to the MMA warp
 // as soon as it is stored, so P.V of keys 0-63 overlaps the exponentials of
 // keys 64-127.  Scores stay in register pairs and use packed fp32 arithmetic.
+// With kPartial, keys outside [kv_lo, kv_hi) get weight 0: the ragged last tile
+// of a segment (kv_lo = 0), or a row's own segment inside a group tile.
 template <bool kPartial, bool kNeg, int D>
-__device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_valid, bool first, float c,
+__device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_lo, int kv_hi, bool first, float c,
                                              uint32_t tS, uint32_t tO, float& m, float& l, float& lr,
                                              uint64_t* p_full_half, int lane) {
-  const float xmax = row_extreme<kPartial, kNeg>(v, kv_valid) * c;  // log2 units
+  const float xmax = row_extreme<kPartial, kNeg>(v, kv_lo, kv_hi) * c;  // log2 units
   bool rescale = false;  // warp-uniform
   float alpha = 1.f;
   if (first) {
@@ -447,13 +546,14 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
         const int i = cc * 16 + k;  // pair index: keys 2i, 2i+1
         uint64_t x = f2_fma(v[i], c2, negm2);
         if (kPartial) {
-          x = f2_pack(2 * i < kv_valid ? f2_lo(x) : -INFINITY, 2 * i + 1 < kv_valid ? f2_hi(x) : -INFINITY);
+          x = f2_pack(2 * i >= kv_lo && 2 * i < kv_hi ? f2_lo(x) : -INFINITY,
+                      2 * i + 1 >= kv_lo && 2 * i + 1 < kv_hi ? f2_hi(x) : -INFINITY);
         }
         const uint64_t pp =
-            (!kPartial && D == 128 && (k & 3) >= 4 - kPolyPairsPer4) ? ex2x2_poly(x, ek) : ex2x2(x);
+            (!kPartial && (k & 3) >= 4 - kPolyPairsPer4<D>) ? ex2x2_poly(x, ek) : ex2x2(x);
         const uint32_t pr = pack_bf16x2_pair(pp);
         su[k & 1] = f2_add(su[k & 1], pp);
-        if (!FwdCfg<D>::kSumColumn) sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
+        if (!FwdCfg<D>::kSumColumn && PA_NORM_ROUNDED_D128) sr[k & 1] = add_bf16x2_as_f32x2(sr[k & 1], pr);
         pk[k] = pr;
       }
       PA_TMEM_ST16(tS + cc * 16, pk);
@@ -484,7 +584,7 @@ __device__ __forceinline__ void softmax_tile(const uint64_t (&v)[64], int kv_val
   }
   const uint64_t su2 = f2_add(su[0], su[1]), sr2 = f2_add(sr[0], sr[1]);
   l += f2_lo(su2) + f2_hi(su2);
-  if (!FwdCfg<D>::kSumColumn) lr += f2_lo(sr2) + f2_hi(sr2);
+  if (!FwdCfg<D>::kSumColumn) lr += PA_NORM_ROUNDED_D128 ? f2_lo(sr2) + f2_hi(sr2) : f2_lo(su2) + f2_hi(su2);
 }
 
 template <int D>
@@ -509,25 +609,43 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
     if (got == -2) ok = false;
     if (got <= 0) break;
     if (tile == 1 && !w.two) continue;
+    // rows of this query tile: tokens [row0, row0 + nrows) of the pack
+    const int32_t row0 = w.beg + w.q0 + tile * (w.n0 ? w.n0 : 128);
+    const int32_t nrows = w.n0 ? (tile ? w.len - w.n0 : w.n0) : w.len - w.q0 - tile * 128;
+    // in a group tile, this row's keys are those of its own segment: [glo, ghi) relative
+    // to the tile (the key tile starts at the query tile's first token)
+    int32_t glo = 0, ghi = nrows;
+    if (w.n0 && t < nrows) {
+      const int32_t tok = row0 + t;
+      int32_t a = w.seg, b = p.batch;  // cu[a] <= tok < cu[b]
+      while (b - a > 1) {
+        const int32_t mid = (a + b) >> 1;
+        if (__ldg(p.cu + mid) <= tok) a = mid; else b = mid;
+      }
+      glo = __ldg(p.cu + a) - row0;
+      ghi = __ldg(p.cu + a + 1) - row0;
+    }
     // l: sum of the fp32 exponentials (gives lse); lr: sum of the same values rounded to
     // bf16, i.e. of the weights the P.V product actually used (normalises the output,
     // so each output row is an exact convex combination of value rows).
     float m = 0.f, l = 0.f, lr = 0.f;
-    for (int32_t j = 0; j < w.nkv; ++j) {
+    for (int32_t j = 0; j < w.kt; ++j) {
       ok = mbar_wait(&bars->s_full[tile], s_ph, wc);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       s_ph ^= 1u;
       tc_fence_after();
       uint64_t r[64];
       tmem_ld128_pairs(tS, r);
-      const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment
+      // keys of this tile that the row sees: the segment's (alone) or its own segment's (group)
+      const int kv_lo = w.n0 ? glo : 0;
+      const int kv_hi = w.n0 ? ghi : w.len - j * 128;
       uint64_t* ph = bars->p_full[tile];
-      if (kv_valid >= 128) {
-        if (c >= 0.f) softmax_tile<false, false, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
-        else softmax_tile<false, true, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+      if (!w.n0 && kv_hi >= 128) {
+        if (c >= 0.f) softmax_tile<false, false, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        else softmax_tile<false, true, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
       } else {
-        if (c >= 0.f) softmax_tile<true, false, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
-        else softmax_tile<true, true, D>(r, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        if (c >= 0.f) softmax_tile<true, false, D>(r, kv_lo, kv_hi, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        else softmax_tile<true, true, D>(r, kv_lo, kv_hi, j == 0, c, tS, tO, m, l, lr, ph, lane);
       }
     }
     if (!ok) break;
@@ -538,10 +656,10 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
     of_ph ^= 1u;
     tc_fence_after();
-    const int32_t row = w.q0 + tile * 128 + t;
-    const bool row_ok = row < w.len;
+    const bool row_ok = t < nrows;
+    const int32_t token = row0 + (row_ok ? t : 0);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
-                                          (static_cast<size_t>(w.beg + (row_ok ? row : 0)) * p.heads + w.head) * D);
+                                          (static_cast<size_t>(token) * p.heads + w.head) * D);
     if (C::kSumColumn) {
       // sum of the bf16 weights, accumulated by the tensor core in O's column d
       uint32_t sc[16];
@@ -570,7 +688,7 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
     if (lane == 0) mbar_arrive(&bars->o_empty[tile]);  // O columns may be overwritten now
     if (row_ok) {
       const float lse2 = m + __log2f(l);
-      p.lse[static_cast<size_t>(w.beg + row) * p.heads + w.head] = lse2 * 0.69314718055994531f;
+      p.lse[static_cast<size_t>(token) * p.heads + w.head] = lse2 * 0.69314718055994531f;
     }
   }
 }

@@ -62,6 +62,7 @@ std::mutex g_mu;
 std::vector<StreamState*> g_states;
 DeviceInfo g_dev[64];
 int g_wait_limit_ms = 4000;
+bool g_short_packing = true;  // pack consecutive short segments into shared tiles (bf16 forward)
 
 // profiling
 bool g_prof_on = false;
@@ -70,16 +71,22 @@ size_t g_prof_used = 0;
 
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Forward workspace: counts (4 int32) and the tile ledger (4 int64, from byte 16) in
+// the first 128 bytes, then order [B], item_start [B+1], the unit descriptors [B]
+// and 3 tensor maps per segment.
 struct WsLayout {
-  size_t counts, order, item_start, maps, total;
+  size_t counts, order, item_start, info, maps, total;
 };
+
+constexpr size_t kStatsOffset = 16;
 
 WsLayout ws_layout(int32_t batch) {
   WsLayout L;
   L.counts = 0;
   L.order = 128;
   L.item_start = align_up(L.order + 4 * static_cast<size_t>(batch), 128);
-  L.maps = align_up(L.item_start + 4 * (static_cast<size_t>(batch) + 1), 128);
+  L.info = align_up(L.item_start + 4 * (static_cast<size_t>(batch) + 1), 128);
+  L.maps = align_up(L.info + 4 * static_cast<size_t>(batch), 128);
   L.total = L.maps + 384 * static_cast<size_t>(batch);
   return L;
 }
@@ -215,9 +222,11 @@ int prof_begin(cudaStream_t stream, cudaEvent_t* ev1) {
 }
 
 // Schedule parameters of a forward call (the template maps are filled by the caller):
-// workspace slices, the pack, pair items (2^8 query rows), the status codes.
+// workspace slices, the pack, pair items (2^8 query rows), the status codes.  With
+// `units`, the scheduler writes unit descriptors (and packs short segments into shared
+// tiles when short-segment packing is on); the FP8 kernel takes one unit per segment.
 pa::SchedParams forward_sched(const int32_t* cu, int32_t* status, uint8_t* ws, const WsLayout& L, int32_t batch,
-                              int32_t total, int32_t heads, int32_t max_seqlen, uint64_t row_bytes) {
+                              int32_t total, int32_t heads, int32_t max_seqlen, uint64_t row_bytes, bool units) {
   pa::SchedParams sp;
   std::memset(&sp, 0, sizeof(sp));
   sp.cu = cu;
@@ -226,6 +235,9 @@ pa::SchedParams forward_sched(const int32_t* cu, int32_t* status, uint8_t* ws, c
   sp.order = reinterpret_cast<int32_t*>(ws + L.order);
   sp.item_start = reinterpret_cast<int32_t*>(ws + L.item_start);
   sp.maps = ws + L.maps;
+  sp.info = units ? reinterpret_cast<int32_t*>(ws + L.info) : nullptr;
+  sp.stats = reinterpret_cast<int64_t*>(ws + L.counts + kStatsOffset);
+  sp.group_short = units && g_short_packing ? 1 : 0;
   sp.row_bytes = row_bytes;
   sp.batch = batch;
   sp.total = total;
@@ -249,8 +261,10 @@ pa::FwdParams forward_params(const pa::SchedParams& sp, void* out, float* lse, f
   fp.order = sp.order;
   fp.item_start = sp.item_start;
   fp.maps = sp.maps;
+  fp.info = sp.info;
   fp.status = sp.status;
   fp.heads = sp.heads;
+  fp.batch = sp.batch;
   fp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   fp.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ms) * 1000000ull;
   fp.err_timeout = PA_ERR_TIMEOUT;
@@ -380,7 +394,7 @@ int pa_varlen_attn_fwd(const void* q, const void* k, const void* v, const int32_
   if ((rc = ensure_workspace(st, L.total)) != PA_OK) return rc;
 
   pa::SchedParams sp = forward_sched(cu_seqlens, st->status, st->ws, L, batch, total_tokens, heads, max_seqlen,
-                                     static_cast<uint64_t>(heads) * head_dim * 2);
+                                     static_cast<uint64_t>(heads) * head_dim * 2, true);
   const void* bases[3] = {q, k, v};
   for (int i = 0; i < 3; ++i) {
     if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
@@ -473,6 +487,7 @@ int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* 
   sp.order = reinterpret_cast<int32_t*>(st->ws + L.order);
   sp.item_start = reinterpret_cast<int32_t*>(st->ws + L.item_start);
   sp.maps = nullptr;
+  sp.stats = reinterpret_cast<int64_t*>(st->ws + L.counts + kStatsOffset);
   sp.batch = batch;
   sp.total = total_tokens;
   sp.heads = heads;
@@ -692,6 +707,35 @@ void pa_release_workspace(void) {
   g_states.clear();
 }
 
+void pa_set_short_packing(int on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_short_packing = on != 0;
+}
+
+int pa_schedule_stats(void* stream_handle, int64_t* out) {
+  if (!out) return PA_ERR_NULL;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  uint8_t* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (StreamState* s : g_states)
+      if (s->device == dev && s->stream == stream) ws = s->ws;
+  }
+  if (!ws) return PA_ERR_NOT_DEVICE;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+  int32_t counts[2];
+  int64_t stats[4];
+  if (cudaMemcpy(counts, ws, sizeof(counts), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(stats, ws + kStatsOffset, sizeof(stats), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PA_ERR_CUDA;
+  out[0] = counts[0];
+  out[1] = counts[1];
+  for (int i = 0; i < 4; ++i) out[2 + i] = stats[i];
+  return PA_OK;
+}
+
 void pa_set_wait_limit_ms(int ms) {
   std::lock_guard<std::mutex> lock(g_mu);
   g_wait_limit_ms = ms < 1 ? 1 : ms;
@@ -775,11 +819,12 @@ int pa_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, cons
   const WsLayout L = ws_layout(batch);
 
   // The status word must start at zero; the schedule kernel rewrites the rest
-  // (counts, work counter, order, item starts, tensor maps) before it is read.
+  // (counts, work counter, order, item starts, unit descriptors, tensor maps)
+  // before it is read.
   if (cudaMemsetAsync(st, 0, sizeof(int32_t), stream) != cudaSuccess) return PA_ERR_CUDA;
 
   pa::SchedParams sp = forward_sched(cu_seqlens, st, ws, L, batch, total_tokens, heads, max_seqlen,
-                                     static_cast<uint64_t>(heads) * head_dim * 2);
+                                     static_cast<uint64_t>(heads) * head_dim * 2, true);
   const void* bases[3] = {q, k, v};
   for (int i = 0; i < 3; ++i) {
     if (!encode_map(&sp.tmpl[i], bases[i], total_tokens, heads, head_dim)) return PA_ERR_CUDA;
@@ -887,7 +932,7 @@ int pa_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8t, cons
 
   const int64_t hd = static_cast<int64_t>(heads) * head_dim;
   pa::SchedParams sp = forward_sched(cu_seqlens, st->status, st->ws, L, batch, total_tokens, heads, max_seqlen,
-                                     static_cast<uint64_t>(hd));
+                                     static_cast<uint64_t>(hd), false);
   if (!encode_u8(&sp.tmpl[0], q8, hd, total_tokens, hd) || !encode_u8(&sp.tmpl[1], k8, hd, total_tokens, hd) ||
       !encode_u8(&sp.tmpl[2], v8t, vt_keys, hd, vt_keys))
     return PA_ERR_CUDA;

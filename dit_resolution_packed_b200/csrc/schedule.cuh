@@ -5,22 +5,43 @@
 //   1. validates cu_seqlens (cu[0] = 0, non-decreasing, cu[B] = T, every
 //      segment <= max_seqlen); on failure it records the status and publishes
 //      an empty work list;
-//   2. orders the non-empty segments longest-first (stable counting sort on the
-//      number of 128-key tiles, i.e. on the per-item cost), so a persistent grid
-//      takes the big items first (longest-processing-time order);
-//   3. publishes, in that order, the first work-item index of every segment;
-//      a segment of L tokens holds heads * ceil(L / 2^rows_log2) items: for the
+//   2. (forward, short-segment packing on) packs runs of consecutive short
+//      segments (at most 128 tokens each) into shared 128-row tiles, two tiles
+//      per unit (see "Short-segment groups" below); every other non-empty
+//      segment is a unit of its own;
+//   3. orders the units longest-first (stable counting sort on the number of
+//      128-key tiles a query tile of the unit meets, i.e. on the per-item cost),
+//      so a persistent grid takes the big items first (longest-processing-time
+//      order);
+//   4. publishes, in that order, the first work-item index of every unit; a
+//      segment of L tokens holds heads * ceil(L / 2^rows_log2) items: for the
 //      forward (rows_log2 = 8) one per (head, pair of 128-row query tiles), for
-//      the backward (rows_log2 = 7) one per (head, 128-key tile);
-//   4. for the forward, writes three tensor maps per segment (q, k, v) whose
-//      base is the segment's first token and whose row extent is L, so that
-//      every TMA tile stops at the segment boundary: loads past it read zeros
-//      and no tile touches another image (maps == nullptr skips this step);
-//      the FP8 variant's transposed V map is cut along its key axis instead.
+//      the backward (rows_log2 = 7) one per (head, 128-key tile); a group of
+//      short segments holds one item per head;
+//   5. for the forward, writes three tensor maps per unit (q, k, v) whose base
+//      is the unit's first token and whose row extent is its token count, so
+//      that every TMA tile stops at the unit's end: loads past it read zeros and
+//      no tile touches an image outside the unit (maps == nullptr skips this
+//      step); the FP8 variant's transposed V map is cut along its key axis;
+//   6. records the tile ledger of the call: 128 x 128 score tiles computed and
+//      useful (query, key) pairs, over all heads.
+//
+// Short-segment groups.  A segment of L <= 128 tokens alone would occupy a whole
+// 128-row query tile and a whole 128-key tile, most of it masked.  Consecutive
+// short segments are instead cut greedily, in packing order, into tiles of at most
+// 128 tokens that hold whole segments; two neighbouring tiles form one unit (a
+// contiguous token range [beg, beg + len) split at n0: tile 0 = [beg, beg + n0),
+// tile 1 = [beg + n0, beg + len)).  Inside a tile the mask is block-diagonal: a
+// query row sees only the keys of its own segment, which lie in its own tile, so
+// tile t meets only key tile t.  To walk the runs in parallel, a run is also cut
+// where a segment starts in a later 1024-token block of the stream than the one
+// before it (at most one part-filled tile per 1024 tokens); each warp walks its
+// own parts.
 //
 // The mask of the method (Mage-Flow page, "Packing + Flash Attention varlen":
 // images attend only to themselves, no padding) is thereby carried entirely by
-// the tensor-map bounds plus the key mask of each segment's last tile.
+// the tensor-map bounds plus the key mask of each segment's last tile (of each
+// row's own segment inside a group tile).
 #pragma once
 #include <cuda.h>
 
@@ -33,16 +54,29 @@ namespace pa {
 constexpr int kSchedThreads = 256;
 constexpr int kSortBuckets = 1024;     // tile counts >= 1023 share the first bucket
 constexpr int kCuInSmem = 4096 + 1;    // cu_seqlens staged in shared memory up to this many entries
+constexpr int kGroupRows = 128;        // tokens of one tile of a short-segment group
+constexpr int kGroupBlockLog2 = 10;    // runs of short segments are also cut at 1024-token blocks
+
+// Unit descriptor of segment i (SchedParams::info): a group head stores its tile
+// split n0 and token count len as n0 | len << 9 (both <= 256); kUnitAlone marks a
+// segment that is a unit by itself, kUnitNone one that is empty or inside a group.
+constexpr int32_t kUnitAlone = -1;
+constexpr int32_t kUnitNone = -2;
+__host__ __device__ constexpr int32_t group_info(int32_t n0, int32_t len) { return n0 | (len << 9); }
+__host__ __device__ constexpr int32_t group_n0(int32_t info) { return info & 0x1ff; }
+__host__ __device__ constexpr int32_t group_len(int32_t info) { return (info >> 9) & 0x1ff; }
 
 struct SchedParams {
   CUtensorMap tmpl[3];     // q, k, v over the whole [T, H*d] matrix (host-encoded)
   const void* base[3];     // q, k, v base pointers
   const int32_t* cu;       // [B+1]
   int32_t* status;         // status word
-  int32_t* counts;         // [0] = work items, [1] = non-empty segments, [2] = work counter (zeroed)
-  int32_t* order;          // [B] segment ids, longest first
-  int32_t* item_start;     // [B+1] first item of each ordered segment
-  uint8_t* maps;           // [B][3] tensor maps, 128 bytes each (nullptr: none)
+  int32_t* counts;         // [0] = work items, [1] = units, [2] = work counter (zeroed)
+  int32_t* order;          // [B] unit ids (a unit's first segment), longest first
+  int32_t* item_start;     // [B+1] first item of each ordered unit
+  uint8_t* maps;           // [B][3] tensor maps, 128 bytes each (nullptr: none); unit i uses slot i
+  int32_t* info;           // [B] unit descriptor per segment (nullptr: every non-empty segment is a unit)
+  int64_t* stats;          // [4] tile ledger: score tiles, useful pairs, groups, grouped segments
   uint64_t row_bytes;      // H * d * 2
   int32_t batch, total, heads, max_seqlen;
   int32_t rows_log2;        // rows of a work item: 2^rows_log2 (8 forward, 7 backward)
@@ -51,6 +85,7 @@ struct SchedParams {
   // per-segment map moves the base to that key and sets the key extent to L
   int32_t v_keys_inner;
   int32_t err_cu, err_max;  // status codes to record
+  int32_t group_short;      // nonzero (and info set): pack consecutive short segments into shared tiles
 };
 
 __device__ __forceinline__ int seg_key(int32_t len) {
@@ -86,6 +121,56 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t v, int64_t* s_wa
   return r;
 }
 
+// ---- short-segment groups (the walk runs on validated cu_seqlens, 0 <= L_i) ----
+
+__device__ __forceinline__ bool seg_short(const int32_t* cu, int i) { return cu[i + 1] - cu[i] <= kGroupRows; }
+
+// Segment i > 0 starts in a later 1024-token block of the stream than segment i - 1.
+__device__ __forceinline__ bool new_block(const int32_t* cu, int i) {
+  return (cu[i - 1] >> kGroupBlockLog2) != (cu[i] >> kGroupBlockLog2);
+}
+
+// A walk starts at every short segment that does not continue the walk of the
+// segment before it.
+__device__ __forceinline__ bool walk_start(const int32_t* cu, int i) {
+  return seg_short(cu, i) && (i == 0 || !seg_short(cu, i - 1) || new_block(cu, i));
+}
+
+// First segment index e in (i, B] that does not join the tile starting at segment i:
+// the end of the pack, a segment that is not short or starts a new walk, or one that
+// would take the tile past kGroupRows tokens.  Called by a whole warp.
+__device__ __forceinline__ int tile_end(const int32_t* cu, int B, int i) {
+  const int lane = threadIdx.x & 31;
+  const int32_t base = cu[i];
+  for (int e0 = i + 1;; e0 += 32) {
+    const int j = e0 + lane;
+    const bool stop = j >= B || !seg_short(cu, j) || new_block(cu, j) || cu[j + 1] - base > kGroupRows;
+    const uint32_t m = __ballot_sync(0xffffffffu, stop);
+    if (m) return e0 + __ffs(m) - 1;
+  }
+}
+
+// Cuts the walk that starts at segment s into pairs of tiles; writes the unit
+// descriptor of every segment it covers.  Called by a whole warp.
+__device__ __forceinline__ void walk_groups(const int32_t* cu, int B, int s, int32_t* info) {
+  const int lane = threadIdx.x & 31;
+  for (int i = s;;) {
+    const int e1 = tile_end(cu, B, i);
+    int e2 = e1;
+    if (e1 < B && seg_short(cu, e1) && !new_block(cu, e1)) e2 = tile_end(cu, B, e1);
+    const int32_t n0 = cu[e1] - cu[i], len = cu[e2] - cu[i];
+    if (lane == 0) info[i] = len > 0 ? group_info(n0, len) : kUnitNone;
+    for (int j = i + 1 + lane; j < e2; j += 32) info[j] = kUnitNone;
+    if (e2 >= B || !seg_short(cu, e2) || new_block(cu, e2)) break;
+    i = e2;
+  }
+}
+
+// Token count a unit's tensor maps cover (0: segment i is not a unit).
+__device__ __forceinline__ int32_t unit_span(int32_t len, int32_t inf) {
+  return inf == kUnitAlone ? len : inf == kUnitNone ? 0 : group_len(inf);
+}
+
 __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid_constant__ SchedParams p) {
   __shared__ int s_bad;
   __shared__ int32_t s_cu_buf[kCuInSmem];
@@ -94,7 +179,9 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   __shared__ int32_t s_keys[kSchedThreads];
   __shared__ int64_t s_warp[32];
   __shared__ int64_t s_total;
+  __shared__ unsigned long long s_ledger[4];
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int B = p.batch;
   // the attention kernel may start its prologue now; it waits for this grid
   // to complete before it reads anything written here
@@ -105,10 +192,11 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   for (int i = tid; staged && i <= B; i += kSchedThreads) s_cu_buf[i] = p.cu[i];
   const int32_t* cu = staged ? s_cu_buf : p.cu;
   if (tid == 0) s_bad = 0;
+  if (tid < 4) s_ledger[tid] = 0;
   for (int b = tid; b < kSortBuckets; b += kSchedThreads) s_hist[b] = 0;
   __syncthreads();
 
-  // 1. validation and histogram of tile counts
+  // 1. validation
   if (tid == 0 && (cu[0] != 0 || cu[B] != p.total)) atomicMax(&s_bad, 2);
   for (int i = tid; i < B; i += kSchedThreads) {
     const int32_t a = cu[i], b = cu[i + 1];
@@ -116,8 +204,6 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       atomicMax(&s_bad, 2);
     } else if (b - a > p.max_seqlen) {
       atomicMax(&s_bad, 1);
-    } else if (b > a) {
-      atomicAdd(&s_hist[seg_key(b - a)], 1);
     }
   }
   __syncthreads();
@@ -127,15 +213,64 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       p.counts[0] = 0;
       p.counts[1] = 0;
       p.counts[2] = 0;
+      if (p.stats)
+        for (int i = 0; i < 4; ++i) p.stats[i] = 0;
     }
     return;
   }
 
-  // 2. per-segment tensor maps: copy the template, then move its base and row extent
+  // 2. units: short-segment groups (each warp walks the runs that start in its
+  // 32-segment chunks), every other non-empty segment alone
+  const bool grouping = p.info != nullptr && p.group_short;
+  if (grouping) {
+    for (int c0 = warp * 32; c0 < B; c0 += kSchedThreads) {
+      const int i = c0 + lane;
+      uint32_t m = __ballot_sync(0xffffffffu, i < B && walk_start(cu, i));
+      while (m) {
+        const int s = c0 + __ffs(m) - 1;
+        m &= m - 1;
+        walk_groups(cu, B, s, p.info);
+      }
+      for (int i2 = c0 + lane; i2 < c0 + 32 && i2 < B; i2 += 32)
+        if (!seg_short(cu, i2)) p.info[i2] = kUnitAlone;
+    }
+  } else if (p.info != nullptr) {
+    for (int i = tid; i < B; i += kSchedThreads) p.info[i] = cu[i + 1] > cu[i] ? kUnitAlone : kUnitNone;
+  }
+  __syncthreads();
+
+  // 3. histogram of the units' sort keys, and the tile ledger
+  {
+    unsigned long long tiles = 0, pairs = 0, groups = 0, grouped = 0;
+    for (int i = tid; i < B; i += kSchedThreads) {
+      const int32_t len = cu[i + 1] - cu[i];
+      const int32_t inf = p.info ? p.info[i] : (len > 0 ? kUnitAlone : kUnitNone);
+      pairs += static_cast<unsigned long long>(len) * static_cast<unsigned long long>(len);
+      if (grouping && len > 0 && len <= kGroupRows) ++grouped;
+      if (inf == kUnitNone) continue;
+      if (inf == kUnitAlone) {
+        const unsigned long long t = static_cast<unsigned long long>((len + 127) >> 7);
+        tiles += t * t;
+        atomicAdd(&s_hist[seg_key(len)], 1);
+      } else {
+        tiles += group_len(inf) > group_n0(inf) ? 2 : 1;
+        ++groups;
+        atomicAdd(&s_hist[1], 1);  // a group's query tile meets one key tile
+      }
+    }
+    atomicAdd(&s_ledger[0], tiles * static_cast<unsigned long long>(p.heads));
+    atomicAdd(&s_ledger[1], pairs * static_cast<unsigned long long>(p.heads));
+    atomicAdd(&s_ledger[2], groups);
+    atomicAdd(&s_ledger[3], grouped);
+  }
+  __syncthreads();
+
+  // 4. per-unit tensor maps: copy the template, then move its base and row extent
   for (int idx = tid; p.maps != nullptr && idx < 3 * B; idx += kSchedThreads) {
     const int s = idx / 3, which = idx - 3 * s;
     const int32_t beg = cu[s], len = cu[s + 1] - beg;
-    if (len <= 0) continue;
+    const int32_t span = p.info ? unit_span(len, p.info[s]) : len;
+    if (span <= 0) continue;
     uint8_t* dst = p.maps + static_cast<size_t>(idx) * 128;
     const uint4* src = reinterpret_cast<const uint4*>(&p.tmpl[which]);
 #pragma unroll
@@ -143,15 +278,15 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     if (which == 2 && p.v_keys_inner) {
       const uint64_t key0 = 16ull * ((static_cast<uint64_t>(beg) + 15) / 16) + 16ull * static_cast<uint64_t>(s);
       tmap_replace_address(dst, static_cast<const uint8_t*>(p.base[2]) + key0);
-      tmap_replace_dim0(dst, static_cast<uint32_t>(len));
+      tmap_replace_dim0(dst, static_cast<uint32_t>(span));
       continue;
     }
     const uint8_t* seg_base = static_cast<const uint8_t*>(p.base[which]) + static_cast<uint64_t>(beg) * p.row_bytes;
     tmap_replace_address(dst, seg_base);
-    tmap_replace_dim1(dst, static_cast<uint32_t>(len));
+    tmap_replace_dim1(dst, static_cast<uint32_t>(span));
   }
 
-  // 3. bucket offsets in descending tile-count order (each thread owns 4 buckets)
+  // 5. bucket offsets in descending key order (each thread owns 4 buckets)
   {
     constexpr int per = kSortBuckets / kSchedThreads;
     int64_t local = 0;
@@ -163,20 +298,22 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       const int b = kSortBuckets - 1 - (tid * per + j);
       s_start[b] = static_cast<int32_t>(off);
       off += s_hist[b];
-      s_hist[b] = 0;  // reused below as the running count of placed segments
+      s_hist[b] = 0;  // reused below as the running count of placed units
     }
   }
   const int32_t n_sorted = static_cast<int32_t>(s_total);
   __syncthreads();
 
-  // 4. stable placement (within a bucket segments keep their packing order) and,
-  // in the same pass, the first work item of every ordered segment
+  // 6. stable placement (within a bucket units keep their packing order) and,
+  // in the same pass, the first work item of every ordered unit
   for (int c0 = 0; c0 < B; c0 += kSchedThreads) {
     const int i = c0 + tid;
     int key = -1;
     if (i < B) {
       const int32_t len = cu[i + 1] - cu[i];
-      if (len > 0) key = seg_key(len);
+      const int32_t inf = p.info ? p.info[i] : (len > 0 ? kUnitAlone : kUnitNone);
+      if (inf == kUnitAlone) key = seg_key(len);
+      else if (inf != kUnitNone) key = 1;
     }
     s_keys[tid] = key;
     __syncthreads();
@@ -199,7 +336,10 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     if (k < n_sorted) {
       const int s = p.order[k];
       const int32_t len = cu[s + 1] - cu[s];
-      items = static_cast<int64_t>(p.heads) * ((static_cast<int64_t>(len) + (1 << p.rows_log2) - 1) >> p.rows_log2);
+      const int32_t inf = p.info ? p.info[s] : kUnitAlone;
+      items = inf == kUnitAlone
+                  ? static_cast<int64_t>(p.heads) * ((static_cast<int64_t>(len) + (1 << p.rows_log2) - 1) >> p.rows_log2)
+                  : static_cast<int64_t>(p.heads);
     }
     const int64_t ex = block_exclusive_scan(items, s_warp, &s_total);
     if (k < n_sorted) p.item_start[k] = static_cast<int32_t>(carry + ex);
@@ -211,6 +351,8 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     p.counts[0] = static_cast<int32_t>(carry);
     p.counts[1] = n_sorted;
     p.counts[2] = 0;
+    if (p.stats)
+      for (int i = 0; i < 4; ++i) p.stats[i] = static_cast<int64_t>(s_ledger[i]);
   }
   fence_tmap_release();
 }

@@ -230,6 +230,39 @@ PA_API int pa_version(void);
 PA_API void pa_release_workspace(void);
 
 /*
+ * pa_set_short_packing -- short-segment packing in pa_varlen_attn_fwd and
+ * pa_varlen_attn_fwd_noalloc (on by default).  A native-resolution pack of small
+ * images (Mage-Flow page, section "Packing + Flash Attention varlen", and its
+ * padding / bucketing / packing table) has many segments of at most 128 tokens.
+ * With packing on, the scheduler cuts runs of consecutive such segments, in
+ * packing order, into shared 128-row tiles that hold whole segments (two tiles
+ * per work item); inside a tile every query row sees only the keys of its own
+ * segment, so the result is the same block-diagonal attention (the wasted block
+ * work of the Fusion page, section 3.5, shrinks).  With packing off every
+ * non-empty segment has tiles of its own.  Both settings compute the same
+ * definition; they differ in the order of nothing but which rows share a tile.
+ * Affects calls enqueued afterwards; thread-safe.
+ */
+PA_API void pa_set_short_packing(int on);
+
+/*
+ * pa_schedule_stats -- the tile ledger of the last call of pa_varlen_attn_fwd,
+ * pa_varlen_attn_fwd_fp8 or pa_varlen_attn_bwd on the calling thread's current
+ * device and `stream` (synchronises `stream`).
+ * Writes 6 values to `out` (host memory):
+ *   out[0] work items, out[1] units (segments alone + groups of short segments;
+ *          the FP8 forward and the backward take every non-empty segment alone),
+ *   out[2] 128 x 128 score tiles computed over all heads,
+ *   out[3] useful (query, key) pairs over all heads = heads * sum_i L_i^2,
+ *   out[4] groups of short segments, out[5] segments inside groups.
+ * Useful pairs / (score tiles * 16384) is the tile utilisation of the call (the
+ * block-level waste account of the Fusion page, section 3.5).  Returns PA_OK,
+ * PA_ERR_NULL (out is NULL), PA_ERR_NOT_DEVICE (no forward call on this
+ * device and stream yet) or PA_ERR_CUDA.  Not for pa_varlen_attn_fwd_noalloc.
+ */
+PA_API int pa_schedule_stats(void* stream, int64_t* out);
+
+/*
  * pa_set_wait_limit_ms -- limit of every pipeline wait inside the kernels, in
  * milliseconds (default 4000).  After the limit a kernel records
  * PA_ERR_TIMEOUT, stops issuing work, drains what it has in flight and returns.

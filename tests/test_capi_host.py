@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 16
+    assert len(names) == len(set(names)) == 18
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -145,3 +145,14 @@ def test_fp8_host_validation_before_any_cuda_call(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="no fallback"):
         pa.load_library(str(tmp_path / "libpackattn.so"))
+
+
+def test_schedule_stats_without_a_call(lib):
+    """The ledger query refuses a NULL output and a (device, stream) pair that has no call yet,
+    without touching a GPU."""
+    out = (ctypes.c_int64 * 6)()
+    assert lib.pa_schedule_stats(None, None) == pa.PA_ERR_NULL
+    rc = lib.pa_schedule_stats(None, out)
+    assert rc in (pa.PA_ERR_NOT_DEVICE, pa.PA_ERR_CUDA)
+    pa.pa_set_short_packing(False)
+    pa.pa_set_short_packing(True)

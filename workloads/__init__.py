@@ -24,6 +24,8 @@ import torch
 PATCH = 16
 _HERE = os.path.dirname(os.path.abspath(__file__))
 CONFIG_NAMES = ("tiny", "mixed", "training", "interactive", "long")
+# packs of the short-segment (HBM-bound) regime, measured beside the configurations above
+SHORT_PACK_NAMES = ("many_short", "thumbnails")
 
 
 def tokens_for_image(h, w, patch=PATCH):
@@ -156,6 +158,11 @@ def sparseattn_worked_example():
     head 1 in dimension 4 + position; then N(0, 0.15) noise of shape (2, 64, 20)
     is added, k equals q, and v ~ N(0, 1) of shape (64, 3) is shared by both heads.
     Random numbers: ``numpy.random.default_rng(7)``, noise drawn before v.
+
+    The construction follows the input lines of the script printed on that page
+    (section 04) in the same order: the seeded draws must come in the page's order
+    to reproduce its printed digits.  The rest of that script (masks, block costs,
+    the result table) is not reproduced here.
 
     Returns fp64 numpy arrays q (2, 64, 20), k (2, 64, 20), v (64, 3) and the
     frame / position index of every token.

@@ -12,6 +12,14 @@ uniform multiples of 16 in [256, 1024], aspect 1:2 to 2:1, about 40k tokens"):
 ``numpy.random.default_rng(s)``; per image h = 16*integers(16, 65) then
 w = 16*integers(16, 65), rejected when max/min > 2, until 16 images; the first
 seed s >= 0 whose total lies in [38000, 42000] is kept.
+
+Two further packs measure the short-segment (HBM-bound) regime with images of the
+same kind at small native resolutions (thumbnails): ``numpy.random.default_rng``
+with the pack seed; per image h = 16*integers(1, n+1) then w = 16*integers(1, n+1),
+rejected when max/min > 2, until the stated number of images:
+  * many_short: 300 images with sides up to 288 px (1..18 patches a side);
+  * thumbnails: 2048 images with sides up to 176 px (1..11 patches a side), so
+    every image fits one 128-row tile (at most 121 tokens).
 """
 import json
 import math
@@ -35,6 +43,18 @@ def _draw_training_images(seed, n_images=16):
     while len(images) < n_images:
         h = PATCH * int(rng.integers(16, 65))
         w = PATCH * int(rng.integers(16, 65))
+        if max(h, w) / min(h, w) > 2:
+            continue
+        images.append([h, w])
+    return images
+
+
+def draw_small_images(seed, n_images, max_patches):
+    rng = np.random.default_rng(seed)
+    images = []
+    while len(images) < n_images:
+        h = PATCH * int(rng.integers(1, max_patches + 1))
+        w = PATCH * int(rng.integers(1, max_patches + 1))
         if max(h, w) / min(h, w) > 2:
             continue
         images.append([h, w])
@@ -66,6 +86,14 @@ def build_configs():
         dict(name="long", description="one 65536-token segment; 512 sampled query rows per head",
              segments=[65536], heads=8, head_dim=64, seed=4,
              sampled_rows=dict(per_head=512, seed_base=1004)),
+    ]
+    cfgs += [
+        dict(name="many_short", description="300 small images, sides uniform multiples of 16 in [16,288], "
+                                            "aspect 1:2..2:1 (short-segment regime)",
+             images=draw_small_images(5, 300, 18), pack_seed=5, heads=24, head_dim=128, seed=5),
+        dict(name="thumbnails", description="2048 thumbnails, sides uniform multiples of 16 in [16,176], "
+                                            "aspect 1:2..2:1 (every image <= 121 tokens)",
+             images=draw_small_images(6, 2048, 11), pack_seed=6, heads=24, head_dim=128, seed=6),
     ]
     for c in cfgs:
         if "images" in c:
