@@ -326,8 +326,9 @@ def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5):
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, pack.cfg["name"])
+    ledger = pa.pa_schedule_stats(stream)  # the tile ledger of the last call
     call_ms = sum(ms) / len(ms)
-    return dict(steps=steps, ms_per_call=call_ms, kernel_ms=kms,
+    return dict(steps=steps, ms_per_call=call_ms, kernel_ms=kms, ledger=ledger,
                 tflops=pack.flops * world / (call_ms * 1e-3) / 1e12,
                 kernel_tflops=pack.flops / (kms * 1e-3) / 1e12,
                 gbs=pack.bytes * world / (call_ms * 1e-3) / 1e9,
@@ -366,6 +367,7 @@ def run_ours(args, world, rank, local):
     # attention kernel alone (for the roofline): the library brackets it with events on its
     # launch stream; the schedule kernel is outside the events
     kern_avg_ms, t_prof = kernel_ms(pa, call, flush, args.steps)
+    head_ledger = pa.pa_schedule_stats(stream)
     clock_rec = clocks.summary(t_region0, t_region1) if clocks else None
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
@@ -574,6 +576,13 @@ def run_ours(args, world, rank, local):
             rec = measure_pack(pa, pk, flush, stream, args, world, device)
             rec.update(tokens=pk.T, segments=len(pk.segs), heads=pk.H, head_dim=pk.d, valid_flops=pk.flops,
                        unique_bytes=pk.bytes)
+            if name in workloads.SHORT_PACK_NAMES or name == "tiny":
+                # the same pack with short-segment packing off: every segment its own tiles
+                pa.pa_set_short_packing(False)
+                try:
+                    rec["packing_off"] = measure_pack(pa, pk, flush, stream, args, world, device)
+                finally:
+                    pa.pa_set_short_packing(True)
             per_config[name] = rec
             del pk
             torch.cuda.empty_cache()
@@ -616,8 +625,12 @@ def run_ours(args, world, rank, local):
         steady["flops_per_sm_cycle"] = flops / (ss_kern_ms * 1e-3) / (ss_clock["sm_mhz"] * 1e6)
     configs_rec, short_rec = {}, {}
     for name, rec in per_config.items():
+        led = rec["ledger"]
         r = {"tokens": rec["tokens"], "segments": rec["segments"], "heads": rec["heads"],
              "head_dim": rec["head_dim"], "steps": rec["steps"], "ms_per_call": rec["ms_per_call"],
+             "tile_ledger": {"score_tiles": led["score_tiles"], "useful_pairs": led["useful_pairs"],
+                             "tile_utilisation": led["tile_utilisation"], "units": led["units"],
+                             "groups": led["groups"], "grouped_segments": led["grouped_segments"]},
              "value": rec["tflops"], "unit": "TFLOP/s", "pct_of_bf16_peak": 100.0 * rec["tflops"] / world / peak_burst,
              "kernel": {"name": head_kernel_name(rec["head_dim"]), "ms": rec["kernel_ms"],
                         "achieved": rec["kernel_tflops"], "frac": rec["kernel_tflops"] / peak_burst,
@@ -629,6 +642,13 @@ def run_ours(args, world, rank, local):
                         "kernel_achieved": rec["kernel_gbs"], "peak": hbm, "unit": "GB/s",
                         "frac": rec["gbs"] / world / hbm, "kernel_frac": rec["kernel_gbs"] / hbm,
                         "peak_source": f"hbm_gbs ({peak_src}, copy bandwidth)"}
+            off = rec.get("packing_off")
+            if off:
+                r["packing_off"] = {"ms_per_call": off["ms_per_call"], "value": off["tflops"], "unit": "TFLOP/s",
+                                    "gbs": off["gbs"], "kernel_gbs": off["kernel_gbs"],
+                                    "tile_utilisation": off["ledger"]["tile_utilisation"],
+                                    "score_tiles": off["ledger"]["score_tiles"]}
+                r["packing_speedup"] = off["ms_per_call"] / rec["ms_per_call"]
             short_rec[name] = r
         else:
             configs_rec[name] = r
@@ -646,6 +666,9 @@ def run_ours(args, world, rank, local):
             peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])),
         "pct_of_bf16_datasheet_dense": 100.0 * value / world / 2250.0,  # vendor figure, not measured here
         "step_ms_p10_p50_p90": [q10, q50, q90],
+        "tile_ledger": {"score_tiles": head_ledger["score_tiles"], "useful_pairs": head_ledger["useful_pairs"],
+                        "tile_utilisation": head_ledger["tile_utilisation"],
+                        "note": "useful (query, key) pairs / (128 x 128 score tiles computed x 16384), all heads"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "peak_source": (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_prof:.2f} s "

@@ -255,7 +255,32 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
     fence_tmap_acquire(mk);
     fence_tmap_acquire(mv);
     const int32_t xcol = w.head * D;
-    const int32_t step = w.n0 ? w.n0 : 128;  // first token of query / key tile 1 within the unit
+    if (w.n0) {
+      // A group of short segments streams its query tiles through the ring too, in the
+      // order Q_0, K_0, V_0 [, Q_1, K_1, V_1] (tile t at the unit's token t * n0), so the
+      // loads of neighbouring items overlap: the only buffer such an item waits for is a
+      // ring slot.
+      const int ntile = w.two ? 2 : 1;
+      for (int t = 0; ok && t < ntile; ++t) {
+        for (int which = 0; which < 3; ++which) {
+          if (!(ok = mbar_wait(&bars->kv_empty[slot], phase ^ 1u, wc))) break;
+          mbar_arrive_expect_tx(&bars->kv_full[slot], C::kTileBytes);
+          armed |= 1u << slot;
+          armed_phase = (armed_phase & ~(1u << slot)) | (phase << slot);
+          uint8_t* dst = smem + C::kOffKV + slot * C::kTileBytes;
+          const void* m = which == 0 ? mq : which == 1 ? mk : mv;
+#pragma unroll
+          for (int cb = 0; cb < C::kColBlocks; ++cb)
+            tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, t * w.n0, &bars->kv_full[slot]);
+          if (++slot == C::kSlots) {
+            slot = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) break;
+      continue;
+    }
     if (!(ok = mbar_wait(&bars->q_empty, (q_round & 1u) ^ 1u, wc))) break;
     mbar_arrive_expect_tx(&bars->q_full, (w.two ? 2u : 1u) * C::kTileBytes);
     q_armed = true;
@@ -264,7 +289,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
     for (int cb = 0; cb < C::kColBlocks; ++cb) {
       tma_load_2d(smem + C::kOffQ + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0, &bars->q_full);
       if (w.two)
-        tma_load_2d(smem + C::kOffQ + C::kTileBytes + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0 + step,
+        tma_load_2d(smem + C::kOffQ + C::kTileBytes + cb * C::kBlockBytes, mq, xcol + cb * 64, w.q0 + 128,
                     &bars->q_full);
     }
     ++q_round;
@@ -279,7 +304,7 @@ __device__ __forceinline__ void run_producer(const FwdParams& p, uint8_t* smem, 
         const void* m = which ? mv : mk;
 #pragma unroll
         for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, j * step, &bars->kv_full[slot]);
+          tma_load_2d(dst + cb * C::kBlockBytes, m, xcol + cb * 64, j * 128, &bars->kv_full[slot]);
         if (++slot == C::kSlots) {
           slot = 0;
           phase ^= 1u;
@@ -365,16 +390,14 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
     if (got != -2 && leader) mbar_arrive(&bars->sched_empty[(sk - 1) & 1]);
     if (got == -2) ok = false;
     if (got <= 0) break;
-    if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
-    ++q_round;
     if (w.n0) {
       // A group of short segments: S_t = Q_t K_t^T and O_t = P_t V_t, tile t meeting only
-      // key tile t.  The ring holds K_0, V_0 [, K_1, V_1] in this order.
+      // key tile t.  The ring holds Q_0, K_0, V_0 [, Q_1, K_1, V_1] in this order.
       const int ntile = w.two ? 2 : 1;
-      int rs[4];
-      uint32_t rp[4];
+      int rs[6];
+      uint32_t rp[6];
 #pragma unroll
-      for (int o = 0; o < 4; ++o) {
+      for (int o = 0; o < 6; ++o) {
         int s2 = slot + o;
         uint32_t ph2 = phase;
         if (s2 >= C::kSlots) {
@@ -387,21 +410,23 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (t == ntile) break;
-        if (!(ok = mbar_wait(&bars->kv_full[rs[2 * t]], rp[2 * t], wc))) break;
+        const int qs = rs[3 * t], ks = rs[3 * t + 1];
+        if (!(ok = mbar_wait(&bars->kv_full[qs], rp[3 * t], wc))) break;
+        if (!(ok = mbar_wait(&bars->kv_full[ks], rp[3 * t + 1], wc))) break;
         tc_fence_after();
-        issue_s<D>(leader, tmem + C::col_s(t), q_addr0 + t * C::kTileBytes, kv_addr0 + rs[2 * t] * C::kTileBytes);
+        issue_s<D>(leader, tmem + C::col_s(t), kv_addr0 + qs * C::kTileBytes, kv_addr0 + ks * C::kTileBytes);
         mma_commit_if(leader, &bars->s_full[t]);
-        mma_commit_if(leader, &bars->kv_empty[rs[2 * t]]);
+        mma_commit_if(leader, &bars->kv_empty[qs]);
+        mma_commit_if(leader, &bars->kv_empty[ks]);
       }
       if (!ok) break;
-      mma_commit_if(leader, &bars->q_empty);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (t == ntile) break;
         if (!(ok = mbar_wait(&bars->o_empty[t], ((oe_ph >> t) & 1u) ^ 1u, wc))) break;
         oe_ph ^= 1u << t;
-        const int vs = rs[2 * t + 1];
-        if (!(ok = mbar_wait(&bars->kv_full[vs], rp[2 * t + 1], wc))) break;
+        const int vs = rs[3 * t + 2];
+        if (!(ok = mbar_wait(&bars->kv_full[vs], rp[3 * t + 2], wc))) break;
         if (!(ok = mbar_wait(&bars->p_full[t][0], (p_ph >> t) & 1u, wc))) break;
         tc_fence_after();
         issue_pv_half<D>(leader, tmem + C::col_o(t), tmem + C::col_s(t), kv_addr0 + vs * C::kTileBytes, ones_addr, 0, false);
@@ -413,14 +438,16 @@ __device__ __forceinline__ void run_mma(const FwdParams& p, uint8_t* smem, Bars*
         mma_commit_if(leader, &bars->kv_empty[vs]);
       }
       if (!ok) break;
-      slot = w.two ? rs[3] + 1 : rs[1] + 1;
-      phase = w.two ? rp[3] : rp[1];
+      slot = w.two ? rs[5] + 1 : rs[2] + 1;
+      phase = w.two ? rp[5] : rp[2];
       if (slot == C::kSlots) {
         slot = 0;
         phase ^= 1u;
       }
       continue;
     }
+    if (!(ok = mbar_wait(&bars->q_full, q_round & 1u, wc))) break;
+    ++q_round;
     int ks = slot;
     if (!(ok = mbar_wait(&bars->kv_full[slot], phase, wc))) break;
     if (++slot == C::kSlots) { slot = 0; phase ^= 1u; }
@@ -609,53 +636,68 @@ __device__ __forceinline__ void run_softmax(const FwdParams& p, uint8_t* smem, B
     if (got == -2) ok = false;
     if (got <= 0) break;
     if (tile == 1 && !w.two) continue;
-    // rows of this query tile: tokens [row0, row0 + nrows) of the pack
-    const int32_t row0 = w.beg + w.q0 + tile * (w.n0 ? w.n0 : 128);
-    const int32_t nrows = w.n0 ? (tile ? w.len - w.n0 : w.n0) : w.len - w.q0 - tile * 128;
-    // in a group tile, this row's keys are those of its own segment: [glo, ghi) relative
-    // to the tile (the key tile starts at the query tile's first token)
-    int32_t glo = 0, ghi = nrows;
-    if (w.n0 && t < nrows) {
-      const int32_t tok = row0 + t;
-      int32_t a = w.seg, b = p.batch;  // cu[a] <= tok < cu[b]
-      while (b - a > 1) {
-        const int32_t mid = (a + b) >> 1;
-        if (__ldg(p.cu + mid) <= tok) a = mid; else b = mid;
-      }
-      glo = __ldg(p.cu + a) - row0;
-      ghi = __ldg(p.cu + a + 1) - row0;
-    }
     // l: sum of the fp32 exponentials (gives lse); lr: sum of the same values rounded to
     // bf16, i.e. of the weights the P.V product actually used (normalises the output,
     // so each output row is an exact convex combination of value rows).
     float m = 0.f, l = 0.f, lr = 0.f;
-    for (int32_t j = 0; j < w.kt; ++j) {
+    uint64_t* ph = bars->p_full[tile];
+    if (w.n0) {
+      // A tile of a group of short segments: one score tile; this row's keys are those of
+      // its own segment, [glo, ghi) relative to the tile (the key tile starts at the query
+      // tile's first token).  Rows past the tile's tokens see [0, nrows) and are not written.
+      const int32_t row0 = w.beg + tile * w.n0;
+      const int32_t nrows = tile ? w.len - w.n0 : w.n0;
+      int32_t glo = 0, ghi = nrows;
+      if (t < nrows) {
+        const int32_t tok = row0 + t;
+        int32_t a = w.seg, b = p.batch;  // cu[a] <= tok < cu[b]
+        while (b - a > 1) {
+          const int32_t mid = (a + b) >> 1;
+          if (__ldg(p.cu + mid) <= tok) a = mid; else b = mid;
+        }
+        glo = __ldg(p.cu + a) - row0;
+        ghi = __ldg(p.cu + a + 1) - row0;
+      }
       ok = mbar_wait(&bars->s_full[tile], s_ph, wc);
-      if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
       s_ph ^= 1u;
       tc_fence_after();
       uint64_t r[64];
       tmem_ld128_pairs(tS, r);
-      // keys of this tile that the row sees: the segment's (alone) or its own segment's (group)
-      const int kv_lo = w.n0 ? glo : 0;
-      const int kv_hi = w.n0 ? ghi : w.len - j * 128;
-      uint64_t* ph = bars->p_full[tile];
-      if (!w.n0 && kv_hi >= 128) {
-        if (c >= 0.f) softmax_tile<false, false, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
-        else softmax_tile<false, true, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
-      } else {
-        if (c >= 0.f) softmax_tile<true, false, D>(r, kv_lo, kv_hi, j == 0, c, tS, tO, m, l, lr, ph, lane);
-        else softmax_tile<true, true, D>(r, kv_lo, kv_hi, j == 0, c, tS, tO, m, l, lr, ph, lane);
+      if (c >= 0.f) softmax_tile<true, false, D>(r, glo, ghi, true, c, tS, tO, m, l, lr, ph, lane);
+      else softmax_tile<true, true, D>(r, glo, ghi, true, c, tS, tO, m, l, lr, ph, lane);
+    } else {
+      for (int32_t j = 0; j < w.nkv; ++j) {
+        ok = mbar_wait(&bars->s_full[tile], s_ph, wc);
+        if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+        s_ph ^= 1u;
+        tc_fence_after();
+        uint64_t r[64];
+        tmem_ld128_pairs(tS, r);
+        const int kv_valid = w.len - j * 128;  // keys of this tile inside the segment
+        if (kv_valid >= 128) {
+          if (c >= 0.f) softmax_tile<false, false, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
+          else softmax_tile<false, true, D>(r, 0, 128, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        } else {
+          if (c >= 0.f) softmax_tile<true, false, D>(r, 0, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+          else softmax_tile<true, true, D>(r, 0, kv_valid, j == 0, c, tS, tO, m, l, lr, ph, lane);
+        }
       }
     }
     if (!ok) break;
 
     // ---- epilogue: O / l -> bf16 -> 16-byte stores of this thread's row (rows past the
-    // segment end are not written); lse from the unrounded sum.
+    // tile's tokens are not written); lse from the unrounded sum.
     ok = mbar_wait(&bars->o_full[tile], of_ph, wc);
     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
     of_ph ^= 1u;
     tc_fence_after();
+    // rows of this query tile: tokens [row0, row0 + nrows) of the pack
+    const int32_t row0 = w.beg + (w.n0 ? tile * w.n0 : w.q0 + tile * 128);
+    const int32_t nrows = w.n0 ? (tile ? w.len - w.n0 : w.n0) : w.len - w.q0 - tile * 128;
     const bool row_ok = t < nrows;
     const int32_t token = row0 + (row_ok ? t : 0);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +

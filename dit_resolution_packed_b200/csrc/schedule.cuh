@@ -152,7 +152,7 @@ __device__ __forceinline__ int tile_end(const int32_t* cu, int B, int i) {
 
 // Cuts the walk that starts at segment s into pairs of tiles; writes the unit
 // descriptor of every segment it covers.  Called by a whole warp.
-__device__ __forceinline__ void walk_groups(const int32_t* cu, int B, int s, int32_t* info) {
+__device__ __forceinline__ void walk_groups(const int32_t* cu, int B, int s, int32_t* __restrict__ info) {
   const int lane = threadIdx.x & 31;
   for (int i = s;;) {
     const int e1 = tile_end(cu, B, i);
@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   __shared__ int32_t s_hist[kSortBuckets];
   __shared__ int32_t s_start[kSortBuckets];
   __shared__ int32_t s_keys[kSchedThreads];
+  __shared__ int32_t s_info_buf[kCuInSmem - 1];
   __shared__ int64_t s_warp[32];
   __shared__ int64_t s_total;
   __shared__ unsigned long long s_ledger[4];
@@ -220,8 +221,10 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   }
 
   // 2. units: short-segment groups (each warp walks the runs that start in its
-  // 32-segment chunks), every other non-empty segment alone
+  // 32-segment chunks), every other non-empty segment alone.  The descriptors are
+  // built in shared memory when the pack is staged there (copied out at the end)
   const bool grouping = p.info != nullptr && p.group_short;
+  int32_t* info = staged ? s_info_buf : p.info;  // working copy (nullptr: computed on the fly)
   if (grouping) {
     for (int c0 = warp * 32; c0 < B; c0 += kSchedThreads) {
       const int i = c0 + lane;
@@ -229,22 +232,25 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       while (m) {
         const int s = c0 + __ffs(m) - 1;
         m &= m - 1;
-        walk_groups(cu, B, s, p.info);
+        walk_groups(cu, B, s, info);
       }
-      for (int i2 = c0 + lane; i2 < c0 + 32 && i2 < B; i2 += 32)
-        if (!seg_short(cu, i2)) p.info[i2] = kUnitAlone;
+      if (i < B && !seg_short(cu, i)) info[i] = kUnitAlone;
     }
-  } else if (p.info != nullptr) {
-    for (int i = tid; i < B; i += kSchedThreads) p.info[i] = cu[i + 1] > cu[i] ? kUnitAlone : kUnitNone;
+  } else if (info != nullptr) {
+    for (int i = tid; i < B; i += kSchedThreads) info[i] = cu[i + 1] > cu[i] ? kUnitAlone : kUnitNone;
   }
   __syncthreads();
+  auto unit_of = [&](int i) -> int32_t {
+    if (info != nullptr) return info[i];
+    return cu[i + 1] > cu[i] ? kUnitAlone : kUnitNone;
+  };
 
   // 3. histogram of the units' sort keys, and the tile ledger
   {
     unsigned long long tiles = 0, pairs = 0, groups = 0, grouped = 0;
     for (int i = tid; i < B; i += kSchedThreads) {
       const int32_t len = cu[i + 1] - cu[i];
-      const int32_t inf = p.info ? p.info[i] : (len > 0 ? kUnitAlone : kUnitNone);
+      const int32_t inf = unit_of(i);
       pairs += static_cast<unsigned long long>(len) * static_cast<unsigned long long>(len);
       if (grouping && len > 0 && len <= kGroupRows) ++grouped;
       if (inf == kUnitNone) continue;
@@ -258,10 +264,19 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
         atomicAdd(&s_hist[1], 1);  // a group's query tile meets one key tile
       }
     }
-    atomicAdd(&s_ledger[0], tiles * static_cast<unsigned long long>(p.heads));
-    atomicAdd(&s_ledger[1], pairs * static_cast<unsigned long long>(p.heads));
-    atomicAdd(&s_ledger[2], groups);
-    atomicAdd(&s_ledger[3], grouped);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+      pairs += __shfl_xor_sync(0xffffffffu, pairs, o);
+      groups += __shfl_xor_sync(0xffffffffu, groups, o);
+      grouped += __shfl_xor_sync(0xffffffffu, grouped, o);
+    }
+    if (lane == 0) {
+      atomicAdd(&s_ledger[0], tiles * static_cast<unsigned long long>(p.heads));
+      atomicAdd(&s_ledger[1], pairs * static_cast<unsigned long long>(p.heads));
+      atomicAdd(&s_ledger[2], groups);
+      atomicAdd(&s_ledger[3], grouped);
+    }
   }
   __syncthreads();
 
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
   for (int idx = tid; p.maps != nullptr && idx < 3 * B; idx += kSchedThreads) {
     const int s = idx / 3, which = idx - 3 * s;
     const int32_t beg = cu[s], len = cu[s + 1] - beg;
-    const int32_t span = p.info ? unit_span(len, p.info[s]) : len;
+    const int32_t span = unit_span(len, unit_of(s));
     if (span <= 0) continue;
     uint8_t* dst = p.maps + static_cast<size_t>(idx) * 128;
     const uint4* src = reinterpret_cast<const uint4*>(&p.tmpl[which]);
@@ -311,7 +326,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     int key = -1;
     if (i < B) {
       const int32_t len = cu[i + 1] - cu[i];
-      const int32_t inf = p.info ? p.info[i] : (len > 0 ? kUnitAlone : kUnitNone);
+      const int32_t inf = unit_of(i);
       if (inf == kUnitAlone) key = seg_key(len);
       else if (inf != kUnitNone) key = 1;
     }
@@ -336,7 +351,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     if (k < n_sorted) {
       const int s = p.order[k];
       const int32_t len = cu[s + 1] - cu[s];
-      const int32_t inf = p.info ? p.info[s] : kUnitAlone;
+      const int32_t inf = unit_of(s);
       items = inf == kUnitAlone
                   ? static_cast<int64_t>(p.heads) * ((static_cast<int64_t>(len) + (1 << p.rows_log2) - 1) >> p.rows_log2)
                   : static_cast<int64_t>(p.heads);
@@ -346,6 +361,8 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
     carry += s_total;
     __syncthreads();
   }
+  // the attention kernel reads the descriptors from global memory
+  for (int i = tid; staged && p.info != nullptr && i < B; i += kSchedThreads) p.info[i] = s_info_buf[i];
   if (tid == 0) {
     p.item_start[n_sorted] = static_cast<int32_t>(carry);
     p.counts[0] = static_cast<int32_t>(carry);
