@@ -33,7 +33,8 @@
 // contiguous token range [beg, beg + len) split at n0: tile 0 = [beg, beg + n0),
 // tile 1 = [beg + n0, beg + len)).  Inside a tile the mask is block-diagonal: a
 // query row sees only the keys of its own segment, which lie in its own tile, so
-// tile t meets only key tile t.  To walk the runs in parallel, a run is also cut
+// tile t meets only key tile t.  A unit that would hold a single segment leaves that
+// segment alone (one tile of its own: nothing to share).  To walk the runs in parallel, a run is also cut
 // where a segment starts in a later 1024-token block of the stream than the one
 // before it (at most one part-filled tile per 1024 tokens); each warp walks its
 // own parts.
@@ -159,7 +160,8 @@ __device__ __forceinline__ void walk_groups(const int32_t* cu, int B, int s, int
     int e2 = e1;
     if (e1 < B && seg_short(cu, e1) && !new_block(cu, e1)) e2 = tile_end(cu, B, e1);
     const int32_t n0 = cu[e1] - cu[i], len = cu[e2] - cu[i];
-    if (lane == 0) info[i] = len > 0 ? group_info(n0, len) : kUnitNone;
+    // a group of one segment gains nothing from sharing: that segment stays a unit alone
+    if (lane == 0) info[i] = len <= 0 ? kUnitNone : e2 == i + 1 ? kUnitAlone : group_info(n0, len);
     for (int j = i + 1 + lane; j < e2; j += 32) info[j] = kUnitNone;
     if (e2 >= B || !seg_short(cu, e2) || new_block(cu, e2)) break;
     i = e2;
@@ -252,7 +254,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(const __grid
       const int32_t len = cu[i + 1] - cu[i];
       const int32_t inf = unit_of(i);
       pairs += static_cast<unsigned long long>(len) * static_cast<unsigned long long>(len);
-      if (grouping && len > 0 && len <= kGroupRows) ++grouped;
+      if (len > 0 && inf != kUnitAlone) ++grouped;  // a non-empty segment inside a group
       if (inf == kUnitNone) continue;
       if (inf == kUnitAlone) {
         const unsigned long long t = static_cast<unsigned long long>((len + 127) >> 7);

@@ -6,7 +6,8 @@ Rules (from the scheduler's description in ``include/packattn.h``, ``pa_set_shor
     consecutive short segments are cut greedily, in packing order, into tiles of at most
     128 tokens holding whole segments; a run is also cut where a segment starts in a later
     1024-token block of the stream than the segment before it;
-  * two neighbouring tiles of a run form one unit (a group), one work item per head;
+  * two neighbouring tiles of a run form one unit (a group), one work item per head; a unit
+    that would hold a single segment leaves that segment alone;
   * every other non-empty segment is a unit of its own with heads * ceil(L / 256) items;
   * score tiles computed: ceil(L/128)^2 per head for a segment alone, one per tile of a group.
 Test infrastructure only; it shares no code with the CUDA path.
@@ -54,7 +55,9 @@ def units(lengths, short_packing=True):
             e1 = tile_end(s)
             e2 = tile_end(e1) if continues(e1) else e1
             n0, ln = cu[e1] - cu[s], cu[e2] - cu[s]
-            if ln > 0:
+            if ln > 0 and e2 == s + 1:
+                out.append(("alone", s, lengths[s]))  # a group of one segment: the segment alone
+            elif ln > 0:
                 out.append(("group", s, n0, ln, list(range(s, e2))))
             if not continues(e2):
                 break
@@ -74,7 +77,7 @@ def ledger(lengths, heads, short_packing=True):
             items += heads
             tiles += heads * (2 if u[3] > u[2] else 1)
             groups += 1
-    grouped = sum(1 for n in lengths if 0 < n <= TILE) if short_packing else 0
+    grouped = sum(1 for u in us if u[0] == "group" for i in u[4] if lengths[i] > 0)
     pairs = heads * sum(int(n) * int(n) for n in lengths)
     return dict(items=items, units=len(us), score_tiles=tiles, useful_pairs=pairs, groups=groups,
                 grouped_segments=grouped)

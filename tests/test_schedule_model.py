@@ -12,9 +12,10 @@ def _check_invariants(lengths):
     seen = {}
     for u in us:
         if u[0] == "alone":
-            assert lengths[u[1]] > sm.TILE
+            assert lengths[u[1]] > 0
             seen[u[1]] = seen.get(u[1], 0) + 1
             continue
+        assert len(u[4]) >= 2  # a group shares its tiles between at least two segments
         _, s, n0, ln, segs = u
         assert segs == list(range(s, s + len(segs)))           # consecutive
         assert all(lengths[j] <= sm.TILE for j in segs)         # short only
@@ -51,12 +52,14 @@ def test_greedy_cut_is_maximal():
     us = _check_invariants(lengths)
     # tile 0 = 60 + 60 (the 10 would make 130), tile 1 = 10 + 100; then 28 (128 would make 156),
     # tile 1 = 128; then 1
-    assert [(g[2], g[3]) for g in us] == [(120, 230), (28, 156), (1, 1)]
+    assert [(g[2], g[3]) for g in us[:2]] == [(120, 230), (28, 156)]
+    assert us[2] == ("alone", 6, 1)  # the last tile holds one segment: it stays alone
 
 
 def test_long_segments_cut_runs():
     us = _check_invariants([50, 50, 300, 20, 20, 129, 0, 7])
     kinds = [(u[0], u[1]) for u in us]
+    # the last run [0, 7] spans two segment indices (one of them empty): a group
     assert kinds == [("group", 0), ("alone", 2), ("group", 3), ("alone", 5), ("group", 6)]
     assert us[-1][3] == 7
 
@@ -68,13 +71,16 @@ def test_block_boundary_cuts_a_run():
     us = _check_invariants(lengths)
     starts = [u[1] for u in us]
     assert 11 in starts
-    assert sum(u[3] for u in us) == 1500
+    assert sum(u[3] if u[0] == "group" else u[2] for u in us) == 1500
+    # the run cut at token 1100 leaves segment 10 (tokens 1000-1099) as the only one of its walk
+    assert ("alone", 10, 100) in us
 
 
 def test_ledger_counts():
     lengths = [0, 5, 0, 130, 0, 0, 257, 0]
     led = sm.ledger(lengths, heads=2)
-    # units: group [0..3) (5 tokens), 130 alone, group [4..6) (empty: no unit), 257 alone, trailing 0: none
+    # units: [0..3) holds the 5-token segment with two empty ones: a group of several
+    # segments; 130 alone, [4..6) empty (no unit), 257 alone, trailing 0: none
     assert led["units"] == 3 and led["groups"] == 1
     assert led["score_tiles"] == 2 * (1 + 4 + 9)
     assert led["items"] == 2 * (1 + 1 + 2)
