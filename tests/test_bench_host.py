@@ -72,3 +72,24 @@ def test_oracle_sample_rate_is_bounded(bench):
     p = workloads.make_inputs(cfg)
     rate, rows, secs, threads = bench.oracle_sample_rate(p, cfg, 0.2)
     assert rate > 0 and rows > 0 and threads >= 1 and secs < 30
+
+
+def test_unique_bytes_of_a_call(bench):
+    # q, k, v read and out written in bf16 (4 tensors x 2 bytes), lse written in fp32
+    assert bench.unique_bytes(10, 3, 128) == 4.0 * 10 * 3 * 128 * 2 + 4.0 * 10 * 3
+    cfg = workloads.load_config("thumbnails")
+    T = sum(cfg["segments"])
+    assert bench.unique_bytes(T, 24, 128) == pytest.approx(2.408e9, rel=1e-3)
+
+
+def test_short_segment_packs_follow_their_recipe():
+    """The frozen small-image packs are what their documented draw produces (sides multiples of
+    16, aspect at most 2, tokens (h/16)(w/16)); every thumbnail fits one 128-row tile."""
+    from workloads import freeze_configs as fc
+    for name, seed, n, max_patches in (("many_short", 5, 300, 18), ("thumbnails", 6, 2048, 11)):
+        cfg = workloads.load_config(name)
+        imgs = fc.draw_small_images(seed, n, max_patches)
+        assert cfg["images"] == imgs
+        assert cfg["segments"] == [workloads.tokens_for_image(h, w) for h, w in imgs]
+        assert all(max(h, w) <= 2 * min(h, w) for h, w in imgs)
+    assert max(workloads.load_config("thumbnails")["segments"]) <= 128
