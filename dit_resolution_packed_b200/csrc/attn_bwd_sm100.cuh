@@ -96,8 +96,8 @@ struct BwdParams {
 struct BwdBars {
   uint64_t kv_full, kv_empty;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t s_full;     // S^T and dP^T of the current query tile are in tensor memory
-  uint64_t pds_full;   // P^T, dS^T stored (tensor memory and shared memory)
+  uint64_t s_full[2];    // S^T and dP^T of query half h of the current tile are in tensor memory
+  uint64_t pds_full[2];  // P^T, dS^T of query half h stored (tensor memory and shared memory)
   uint64_t dq_full, dq_empty;
   uint64_t dkv_full, dkv_empty;
   uint64_t stage_full, stage_empty;  // the per-query -lse2, -D*scale staging of the elementwise warps
@@ -227,10 +227,11 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, uint8_t* smem, 
 
 // ------------------------------------------------------------------ MMA issuer
 // A (M x K) from shared memory K-major, B (N x K) K-major: a score-like product
-// over d (S^T = K Q^T, dP^T = V dO^T).  N = 128.
-template <int D>
+// over d (S^T = K Q^T with N = 128; dP^T = V dO^T one half of the queries at a time,
+// N = 64, B starting at the half's first row: 64 rows of 128 bytes into each block).
+template <int D, int N = 128>
 __device__ __forceinline__ void bwd_issue_kmajor(uint32_t issue, uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+  constexpr uint32_t idesc = idesc_bf16_f32(128, N, false);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
   const uint32_t a0 = sdesc_sw128_lo(a_addr, 16), b0 = sdesc_sw128_lo(b_addr, 16);
 #pragma unroll
@@ -241,15 +242,16 @@ __device__ __forceinline__ void bwd_issue_kmajor(uint32_t issue, uint32_t d_tmem
 }
 
 // D (+)= A B with A (128 rows x 128 along K) bf16 in tensor memory and B (K = 128
-// token rows x N = d) MN-major in shared memory: dV += P^T dO, dK += dS^T Q.
-template <int D>
+// token rows x N = d) MN-major in shared memory: dV += P^T dO, dK += dS^T Q.  Only the
+// K steps [K0, K1) of 16 query rows each: half h of the queries is steps [4h, 4h + 4).
+template <int D, int K0, int K1>
 __device__ __forceinline__ void bwd_issue_tmem_a(uint32_t issue, uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr,
                                                  bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, true);
   constexpr uint32_t hi = sdesc_sw128_hi(1024);
   const uint32_t b0 = sdesc_sw128_lo(b_addr, BwdCfg<D>::kBlockBytes);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
+  for (int kk = K0; kk < K1; ++kk)
     mma_bf16_ts_lo_if(issue, d_tmem, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), hi, idesc,
                       (accumulate || kk > 0) ? 1u : 0u);
 }
@@ -300,27 +302,36 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
         dqe_ph ^= 1u;
         tc_fence_after();
       }
-      bwd_issue_kmajor<D>(leader, tmem + C::kColB, v_addr, do_addr0 + cur * C::kTileBytes);
-      mma_commit_if(leader, &bars->s_full);
-      if (!(ok = mbar_wait(&bars->pds_full, pds_ph, wc))) break;
-      pds_ph ^= 1u;
+      // dP^T in two halves of 64 queries, so the elementwise pass starts on the first
+      bwd_issue_kmajor<D, 64>(leader, tmem + C::kColB, v_addr, do_addr0 + cur * C::kTileBytes);
+      mma_commit_if(leader, &bars->s_full[0]);
+      bwd_issue_kmajor<D, 64>(leader, tmem + C::kColB + 64, v_addr, do_addr0 + cur * C::kTileBytes + 64 * 128);
+      mma_commit_if(leader, &bars->s_full[1]);
+      if (!(ok = mbar_wait(&bars->pds_full[0], pds_ph, wc))) break;
       tc_fence_after();
       if (i == 0 && dkv_pending) {  // the previous item's dK, dV have been read
         if (!(ok = mbar_wait(&bars->dkv_empty, dkve_ph, wc))) break;
         dkve_ph ^= 1u;
         tc_fence_after();
       }
-      bwd_issue_tmem_a<D>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
-      bwd_issue_tmem_a<D>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
+      // the first half's dV, dK run while the elementwise warps compute the second half
+      bwd_issue_tmem_a<D, 0, 4>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
+      bwd_issue_tmem_a<D, 0, 4>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
+      if (!(ok = mbar_wait(&bars->pds_full[1], pds_ph, wc))) break;
+      pds_ph ^= 1u;
+      tc_fence_after();
+      // dK's second half reads dS^T from tensor memory B before dQ (d = 128) overwrites it
+      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, true);
       if (C::kOwnDq && dq_pending) {  // dQ's own columns: the previous partial has been read
         if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
         dqe_ph ^= 1u;
         tc_fence_after();
       }
-      // dQ before the next S^T, so that its read-out overlaps that MMA
+      // dQ before dV's second half and the next S^T, so that its read-out overlaps both
       bwd_issue_dq<D>(leader, tmem + C::kColDQ, ds_addr, k_addr);
       mma_commit_if(leader, &bars->dq_full);
       dq_pending = true;
+      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, true);
       mma_commit_if(leader, &bars->qd_empty[cur]);
       if (++qslot == 2) {
         qslot = 0;
@@ -387,19 +398,22 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
       ok = mbar_wait(&bars->stage_full, st_ph, wc);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       st_ph ^= 1u;
-      ok = mbar_wait(&bars->s_full, s_ph, wc);
+      ok = mbar_wait(&bars->s_full[0], s_ph, wc);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-      s_ph ^= 1u;
       tc_fence_after();
       // 32 query columns per chunk; the loads of chunk ch + 1 are in flight while chunk ch
-      // is computed (they read columns 32(ch+1).., the stores of chunk ch write 16ch..16ch+15)
+      // is computed (they read columns 32(ch+1).., the stores of chunk ch write 16ch..16ch+15).
+      // Queries [0, 64) (chunks 0, 1) and [64, 128) (chunks 2, 3) are handed to the MMA warp
+      // separately; dP^T of the second half is read only after its own barrier.
       uint32_t sbuf[2][32], dbuf[2][32];
       PA_TMEM_LD32(tA, sbuf[0]);
       PA_TMEM_LD32(tB, dbuf[0]);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         tmem_wait_ld();
-        if (ch < 3) {
+        if (ch == 1) {
+          PA_TMEM_LD32(tA + 64, sbuf[0]);
+        } else if (ch < 3) {
           PA_TMEM_LD32(tA + 32 * (ch + 1), sbuf[(ch + 1) & 1]);
           PA_TMEM_LD32(tB + 32 * (ch + 1), dbuf[(ch + 1) & 1]);
         }
@@ -428,15 +442,25 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
           *reinterpret_cast<uint4*>(blk + ((c ^ (t & 7)) << 4)) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
+        if (ch & 1) {
+          tmem_wait_st();
+          fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars->pds_full[ch >> 1]);
+            if (ch == 3) mbar_arrive(&bars->stage_empty);
+          }
+          if (ch == 1) {
+            ok = mbar_wait(&bars->s_full[1], s_ph, wc);
+            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            tc_fence_after();
+            PA_TMEM_LD32(tB + 64, dbuf[0]);
+          }
+        }
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars->pds_full);
-        mbar_arrive(&bars->stage_empty);
-      }
+      if (!ok) break;
+      s_ph ^= 1u;
     }
     if (!ok) break;
   }
@@ -540,8 +564,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       mbar_init(&bars->sched_full[s], 1);
       mbar_init(&bars->sched_empty[s], 9);  // the MMA warp + one lane of each of 8 warps
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->pds_full, 4);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars->s_full[h], 1);
+      mbar_init(&bars->pds_full[h], 4);
+    }
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 4);
     mbar_init(&bars->dkv_full, 1);
