@@ -612,47 +612,81 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   }
 }
 
-// D = dout . out per (token, head) and lse * log2(e), both written head-major [H][T].
-// One warp per (token, head) row.
+// D = dout . out per (token, head) and lse * log2(e), both written head-major [H][T];
+// the same launch zeroes the fp32 dq accumulator (acc_n4 float4).  A group of d/8
+// lanes takes one (token, head) row with 16-byte loads; each warp takes 8 rows.
+constexpr int kPrepRowsPerWarp = 8;
 template <int D>
 __global__ void bwd_prep_kernel(const uint16_t* __restrict__ out, const uint16_t* __restrict__ dout,
                                 const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
-                                int32_t total, int32_t heads) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+                                float4* __restrict__ acc, int64_t acc_n4, int32_t total, int32_t heads) {
+  constexpr int kLanes = D / 8;                          // lanes per row
+  constexpr int kIter = kPrepRowsPerWarp * kLanes / 32;  // loads per lane and tensor
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = gtid; i < acc_n4; i += nthreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   const int lane = threadIdx.x & 31;
-  if (row >= static_cast<int64_t>(total) * heads) return;
-  const int32_t tok = static_cast<int32_t>(row / heads), h = static_cast<int32_t>(row - static_cast<int64_t>(tok) * heads);
-  constexpr int kPer = D / 32;  // bf16 elements per lane
-  const uint16_t* o = out + row * D + lane * kPer;
-  const uint16_t* g = dout + row * D + lane * kPer;
-  float acc = 0.f;
+  const int sub = lane / kLanes, col = lane % kLanes;
+  const int64_t nrows = static_cast<int64_t>(total) * heads;
+  const int64_t row0 = (gtid >> 5) * kPrepRowsPerWarp;
+  uint4 a[kIter], g[kIter];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e)
-    acc += __uint_as_float(static_cast<uint32_t>(o[e]) << 16) * __uint_as_float(static_cast<uint32_t>(g[e]) << 16);
+  for (int it = 0; it < kIter; ++it) {
+    const int64_t row = row0 + it * (32 / kLanes) + sub;
+    a[it] = g[it] = make_uint4(0u, 0u, 0u, 0u);
+    if (row < nrows) {
+      a[it] = __ldg(reinterpret_cast<const uint4*>(out + row * D) + col);
+      g[it] = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + col);
+    }
+  }
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
-    const size_t hi = static_cast<size_t>(h) * total + tok;
-    delta[hi] = acc;
-    lse2[hi] = lse[row] * 1.4426950408889634f;
+  for (int it = 0; it < kIter; ++it) {
+    const uint32_t av[4] = {a[it].x, a[it].y, a[it].z, a[it].w};
+    const uint32_t gv[4] = {g[it].x, g[it].y, g[it].z, g[it].w};
+    float acc_d = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc_d += __uint_as_float(av[e] << 16) * __uint_as_float(gv[e] << 16);
+      acc_d += __uint_as_float(av[e] & 0xffff0000u) * __uint_as_float(gv[e] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int s = kLanes / 2; s > 0; s >>= 1) acc_d += __shfl_xor_sync(0xffffffffu, acc_d, s);
+    const int64_t row = row0 + it * (32 / kLanes) + sub;
+    if (col == 0 && row < nrows) {
+      const int32_t tok = static_cast<int32_t>(row / heads), h = static_cast<int32_t>(row - static_cast<int64_t>(tok) * heads);
+      const size_t hi = static_cast<size_t>(h) * total + tok;
+      delta[hi] = acc_d;
+      lse2[hi] = lse[row] * 1.4426950408889634f;
+    }
   }
 }
 
-// dq [T, H, d] bf16 from the fp32 accumulator [H][d/4][T] x 4; one thread per float4.
+// dq [T, H, d] bf16 from the fp32 accumulator [H][d/4][T] x 4.  One block per (32
+// tokens, head): the 32 x d/4 float4 are read token-fastest (512 contiguous bytes per
+// warp), packed to bf16 in shared memory and written as whole rows, 16 bytes per thread.
 template <int D>
-__global__ void bwd_dq_convert_kernel(const float4* __restrict__ acc, uint16_t* __restrict__ dq, int32_t total,
-                                      int32_t heads) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(total) * heads * (D / 4);
-  if (idx >= n) return;
-  const int32_t tok = static_cast<int32_t>(idx % total);
-  const int64_t hc = idx / total;  // h * (D/4) + c4
-  const int32_t h = static_cast<int32_t>(hc / (D / 4)), c4 = static_cast<int32_t>(hc % (D / 4));
-  const float4 v = acc[idx];
-  uint2 pk;
-  pk.x = pack_bf16x2(v.x, v.y);
-  pk.y = pack_bf16x2(v.z, v.w);
-  *reinterpret_cast<uint2*>(dq + (static_cast<size_t>(tok) * heads + h) * D + c4 * 4) = pk;
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float4* __restrict__ acc, uint16_t* __restrict__ dq,
+                                                             int32_t total, int32_t heads) {
+  constexpr int kC4 = D / 4;
+  constexpr int kStride = kC4 * 8 + 16;  // bytes per token row in shared memory (16-byte aligned)
+  constexpr int kChunks = D / 8;         // 16-byte chunks per bf16 row
+  __shared__ __align__(16) uint8_t tile[32 * kStride];
+  const int32_t h = static_cast<int32_t>(blockIdx.x % static_cast<uint32_t>(heads));
+  const int32_t t0 = static_cast<int32_t>(blockIdx.x / static_cast<uint32_t>(heads)) * 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t tok = t0 + lane;
+  for (int c4 = warp; c4 < kC4; c4 += 8) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tok < total) v = __ldcs(acc + (static_cast<size_t>(h) * kC4 + c4) * total + tok);
+    *reinterpret_cast<uint2*>(tile + lane * kStride + c4 * 8) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < 32 * kChunks; j += 256) {
+    const int r = j / kChunks, c = j % kChunks;
+    if (t0 + r < total)
+      *reinterpret_cast<uint4*>(dq + (static_cast<size_t>(t0 + r) * heads + h) * D + c * 8) =
+          *reinterpret_cast<const uint4*>(tile + r * kStride + c * 16);
+  }
 }
 
 }  // namespace pa

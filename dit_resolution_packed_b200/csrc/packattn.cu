@@ -467,16 +467,20 @@ int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* 
   float* dq_acc = reinterpret_cast<float*>(st->ws + L.dq_acc);
   const size_t rows = static_cast<size_t>(total_tokens) * heads;
 
-  if (cudaMemsetAsync(dq_acc, 0, 4 * rows * static_cast<size_t>(head_dim), stream) != cudaSuccess) return PA_ERR_CUDA;
-  const unsigned prep_blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  // one launch: D and lse * log2(e), and the zeroed dq accumulator
+  const int64_t acc_n4 = static_cast<int64_t>(rows) * (head_dim / 4);
+  const size_t prep_warps = (rows + pa::kPrepRowsPerWarp - 1) / pa::kPrepRowsPerWarp;
+  const unsigned prep_blocks = static_cast<unsigned>((prep_warps * 32 + 255) / 256);
   if (head_dim == 128)
     pa::bwd_prep_kernel<128><<<prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
                                                             static_cast<const uint16_t*>(dout), lse, delta, lse2,
-                                                            total_tokens, heads);
+                                                            reinterpret_cast<float4*>(dq_acc), acc_n4, total_tokens,
+                                                            heads);
   else
     pa::bwd_prep_kernel<64><<<prep_blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(out),
                                                            static_cast<const uint16_t*>(dout), lse, delta, lse2,
-                                                           total_tokens, heads);
+                                                           reinterpret_cast<float4*>(dq_acc), acc_n4, total_tokens,
+                                                           heads);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
 
   pa::SchedParams sp;
@@ -534,8 +538,7 @@ int pa_varlen_attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (ev1) cudaEventRecord(ev1, stream);
 
-  const size_t n4 = rows * static_cast<size_t>(head_dim / 4);
-  const unsigned conv_blocks = static_cast<unsigned>((n4 + 255) / 256);
+  const unsigned conv_blocks = static_cast<unsigned>(((static_cast<size_t>(total_tokens) + 31) / 32) * heads);
   if (head_dim == 128)
     pa::bwd_dq_convert_kernel<128><<<conv_blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(dq_acc),
                                                                   static_cast<uint16_t*>(dq), total_tokens, heads);
