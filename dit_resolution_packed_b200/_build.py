@@ -34,13 +34,16 @@ def nvcc_command(out=LIB, extra=()):
             *extra, "-o", out] + [os.path.join(CSRC, f) for f in SOURCES]
 
 
-# The attention kernels split their register pool with setmaxnreg; the split is
-# only valid if every attention kernel is compiled at exactly this count.
+# The forward kernels split their register pool with setmaxnreg; the split is
+# only valid if they are compiled at exactly this count.  The backward kernel runs
+# 16 warps at 128 registers each (the whole register file) without a split.
 LAUNCH_REGS = 168
+BWD_MAX_REGS = 128
 
 
 def _check_registers(ptxas_log):
-    """Fails the build unless each attention kernel uses exactly LAUNCH_REGS registers."""
+    """Fails the build unless each forward attention kernel uses exactly LAUNCH_REGS
+    registers and the backward kernel at most BWD_MAX_REGS."""
     kernel = None
     seen = 0
     for line in ptxas_log.splitlines():
@@ -51,7 +54,10 @@ def _check_registers(ptxas_log):
         m = re.search(r"Used (\d+) registers", line)
         if m and kernel and any(n in kernel for n in ("attn_fwd_kernel", "attn_fwd_fp8_kernel", "attn_bwd_kernel")):
             regs = int(m.group(1))
-            if regs != LAUNCH_REGS:
+            if "attn_bwd_kernel" in kernel:
+                if regs > BWD_MAX_REGS:
+                    raise RuntimeError(f"{kernel}: {regs} registers, at most {BWD_MAX_REGS} for 16 warps")
+            elif regs != LAUNCH_REGS:
                 raise RuntimeError(f"{kernel}: {regs} registers, expected {LAUNCH_REGS} for the register split")
             seen += 1
     if seen == 0:

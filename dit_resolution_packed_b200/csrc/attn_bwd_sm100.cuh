@@ -28,13 +28,14 @@
 // [T, H*d] matrix; past T the load reads zeros) and masked: a query past the
 // end has lse = +inf (so P = 0) and D = 0; a key past the end gets P = dS = 0.
 //
-// CTA layout, 12 warps:
-//   warps 0-3  elementwise: P^T and dS^T of one query tile (one thread per key row)
-//   warps 4-7  dQ partial -> fp32 reductions (one thread per query row); dK, dV
-//              epilogue at the end of the item (one thread per key row)
+// CTA layout, 16 warps (128 registers each; no register split):
+//   warps 0-3, 4-7  two elementwise warpgroups, one per half of the query tile: P^T
+//              and dS^T of its 64 queries (one thread per key row)
 //   warp 8     TMA producer (K, V once per item; Q, dO through a two-slot ring)
 //   warp 9     tensor-memory owner and MMA issuer (whole warp, one elected lane issues)
-//   warps 10-11 idle (they complete the third warpgroup for the register split)
+//   warps 10-11 idle
+//   warps 12-15 dQ partial -> fp32 reductions (one thread per query row); dK, dV
+//              epilogue at the end of the item (one thread per key row)
 #pragma once
 #include <cuda.h>
 
@@ -44,11 +45,9 @@
 
 namespace pa {
 
-constexpr int kBwdThreads = 384;
-constexpr int kBwdLaunchRegs = 168;
-constexpr int kBwdMathRegs = 216;
-constexpr int kBwdControlRegs = 72;
-static_assert(2 * 128 * kBwdMathRegs + 128 * kBwdControlRegs <= kBwdThreads * kBwdLaunchRegs, "register split");
+// 16 warps at 128 registers each (the whole register file): every role fits, so there is
+// no register split between the warpgroups.
+constexpr int kBwdThreads = 512;
 
 template <int D>
 struct BwdCfg {
@@ -64,7 +63,7 @@ struct BwdCfg {
   static constexpr int kOffDS = kOffDO + 2 * kTileBytes;  // dS^T: 128 keys x 128 queries bf16, 2 blocks
   static constexpr int kOffStage = kOffDS + 2 * kBlockBytes;  // -lse2 and -D*scale of the 128 queries
   static constexpr int kOffBar = kOffStage + 2 * 128 * 4;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + 1024 for base alignment
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // + 1024 for base alignment
   static constexpr uint32_t kTmemCols = 512;
   // tensor memory: A [0,128) S^T then P^T; B [128,256) dP^T, dS^T (and dQ at d = 128);
   // dV [256, 256+d); dK [256+d, 256+2d); at d = 64 dQ has its own columns [384, 448),
@@ -98,16 +97,16 @@ struct BwdBars {
   uint64_t qd_full[2], qd_empty[2];
   uint64_t s_full[2];    // S^T and dP^T of query half h of the current tile are in tensor memory
   uint64_t pds_full[2];  // P^T, dS^T of query half h stored (tensor memory and shared memory)
-  uint64_t dq_full, dq_empty;
+  uint64_t dq_full, dq_empty[2];  // dQ in tensor memory; its column halves read out
   uint64_t dkv_full, dkv_empty;
-  uint64_t stage_full, stage_empty;  // the per-query -lse2, -D*scale staging of the elementwise warps
+  uint64_t stage_full[2], stage_empty[2];  // per warpgroup: its queries' -lse2, -D*scale staging
   uint64_t sched_full[2], sched_empty[2];
   uint64_t drain;
   int32_t sched_item[2][8];  // seg, beg, len, head, k0, n query tiles, -, id; seg < 0 = done
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(BwdBars) <= 256, "backward barrier block");
+static_assert(sizeof(BwdBars) <= 512, "backward barrier block");
 
 struct BwdItem {
   int32_t seg, beg, len, head, k0, nq, id;
@@ -297,14 +296,19 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
     bwd_issue_kmajor<D>(leader, tmem + C::kColA, k_addr, q_addr0 + qslot * C::kTileBytes);
     for (int32_t i = 0; i < w.nq; ++i) {
       const int cur = qslot;
-      if (!C::kOwnDq && dq_pending) {  // tensor memory B: the previous dQ partial has been read
-        if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
+      // dP^T in two halves of 64 queries, one per elementwise warpgroup; at d = 128 each
+      // half reuses the tensor-memory columns of one half of the previous dQ partial
+      if (!C::kOwnDq && dq_pending) {
+        if (!(ok = mbar_wait(&bars->dq_empty[0], dqe_ph, wc))) break;
+        tc_fence_after();
+      }
+      bwd_issue_kmajor<D, 64>(leader, tmem + C::kColB, v_addr, do_addr0 + cur * C::kTileBytes);
+      mma_commit_if(leader, &bars->s_full[0]);
+      if (!C::kOwnDq && dq_pending) {
+        if (!(ok = mbar_wait(&bars->dq_empty[1], dqe_ph, wc))) break;
         dqe_ph ^= 1u;
         tc_fence_after();
       }
-      // dP^T in two halves of 64 queries, so the elementwise pass starts on the first
-      bwd_issue_kmajor<D, 64>(leader, tmem + C::kColB, v_addr, do_addr0 + cur * C::kTileBytes);
-      mma_commit_if(leader, &bars->s_full[0]);
       bwd_issue_kmajor<D, 64>(leader, tmem + C::kColB + 64, v_addr, do_addr0 + cur * C::kTileBytes + 64 * 128);
       mma_commit_if(leader, &bars->s_full[1]);
       if (!(ok = mbar_wait(&bars->pds_full[0], pds_ph, wc))) break;
@@ -314,16 +318,17 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
         dkve_ph ^= 1u;
         tc_fence_after();
       }
-      // the first half's dV, dK run while the elementwise warps compute the second half
+      // the first half's dV, dK run while the second warpgroup finishes its half
       bwd_issue_tmem_a<D, 0, 4>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, i > 0);
       bwd_issue_tmem_a<D, 0, 4>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, i > 0);
       if (!(ok = mbar_wait(&bars->pds_full[1], pds_ph, wc))) break;
       pds_ph ^= 1u;
       tc_fence_after();
       // dK's second half reads dS^T from tensor memory B before dQ (d = 128) overwrites it
-      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDK, tmem + C::kColB, q_addr0 + cur * C::kTileBytes, true);
+      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDK, tmem + C::kColB + 32, q_addr0 + cur * C::kTileBytes, true);
       if (C::kOwnDq && dq_pending) {  // dQ's own columns: the previous partial has been read
-        if (!(ok = mbar_wait(&bars->dq_empty, dqe_ph, wc))) break;
+        if (!(ok = mbar_wait(&bars->dq_empty[0], dqe_ph, wc))) break;
+        if (!(ok = mbar_wait(&bars->dq_empty[1], dqe_ph, wc))) break;
         dqe_ph ^= 1u;
         tc_fence_after();
       }
@@ -331,7 +336,7 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
       bwd_issue_dq<D>(leader, tmem + C::kColDQ, ds_addr, k_addr);
       mma_commit_if(leader, &bars->dq_full);
       dq_pending = true;
-      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDV, tmem + C::kColA, do_addr0 + cur * C::kTileBytes, true);
+      bwd_issue_tmem_a<D, 4, 8>(leader, tmem + C::kColDV, tmem + C::kColA + 32, do_addr0 + cur * C::kTileBytes, true);
       mma_commit_if(leader, &bars->qd_empty[cur]);
       if (++qslot == 2) {
         qslot = 0;
@@ -354,17 +359,21 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
 }
 
 // ------------------------------------------------------------------ elementwise: P^T, dS^T
+// Warpgroup h (warps 4h .. 4h+3) computes P^T and dS^T of queries [64h, 64h + 64) of
+// every tile, one thread per key row, in units of 16 query columns (the loads of unit
+// u + 1 in flight while unit u is computed).  They go to tensor-memory columns
+// [64h, 64h + 32) of A and B: each warpgroup reads and writes only its own 64 columns.
 template <int D>
 __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* smem, BwdBars* bars, const WaitCtl& wc,
-                                                uint32_t tmem) {
+                                                uint32_t tmem, int h) {
   using C = BwdCfg<D>;
   const int t = threadIdx.x & 127;  // key row of the tile (tensor-memory lane)
   const int lane = threadIdx.x & 31;
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
-  const uint32_t tA = tmem + lane_base + C::kColA;
-  const uint32_t tB = tmem + lane_base + C::kColB;
+  const uint32_t tA = tmem + lane_base + C::kColA + 64 * h;
+  const uint32_t tB = tmem + lane_base + C::kColB + 64 * h;
   float* stage = reinterpret_cast<float*>(smem + C::kOffStage);  // [0,128): -lse2, [128,256): -D*scale
-  uint8_t* ds_row = smem + C::kOffDS + t * 128;
+  uint8_t* ds_blk = smem + C::kOffDS + h * C::kBlockBytes + t * 128;
   const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
   const uint64_t sc2 = f2_pack(p.scale, p.scale);
   const uint64_t zero2 = 0;
@@ -379,101 +388,94 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
     const bool key_ok = t < w.len - w.k0;
     bool ok = true;
     for (int32_t i = 0; i < w.nq; ++i) {
-      // the 128 queries' -lse2 and -D*scale (+inf lse past the segment end: P = 0)
-      const int32_t qrow = i * 128 + t;
+      // this half's 64 queries' -lse2 and -D*scale (+inf lse past the segment end: P = 0)
+      const int32_t qh = i * 128 + 64 * h + (t & 63);
       float nl = -INFINITY, nd = 0.f;
-      if (qrow < w.len) {
-        const size_t hi = static_cast<size_t>(w.head) * p.total + w.beg + qrow;
+      if (t < 64 && qh < w.len) {
+        const size_t hi = static_cast<size_t>(w.head) * p.total + w.beg + qh;
         nl = -__ldg(p.lse2 + hi);
         nd = -__ldg(p.delta + hi) * p.scale;
       }
       // (bounded mbarrier waits, not named barriers: a warp that gives up must not
       // leave the others blocked)
-      ok = mbar_wait(&bars->stage_empty, st_ph ^ 1u, wc);  // all warps are done with the last stage
+      ok = mbar_wait(&bars->stage_empty[h], st_ph ^ 1u, wc);  // all warps are done with the last stage
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-      stage[t] = nl;
-      stage[128 + t] = nd;
+      if (t < 64) {
+        stage[64 * h + t] = nl;
+        stage[128 + 64 * h + t] = nd;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->stage_full);
-      ok = mbar_wait(&bars->stage_full, st_ph, wc);
+      if (lane == 0) mbar_arrive(&bars->stage_full[h]);
+      ok = mbar_wait(&bars->stage_full[h], st_ph, wc);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       st_ph ^= 1u;
-      ok = mbar_wait(&bars->s_full[0], s_ph, wc);
+      ok = mbar_wait(&bars->s_full[h], s_ph, wc);
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+      s_ph ^= 1u;
       tc_fence_after();
-      // 32 query columns per chunk; the loads of chunk ch + 1 are in flight while chunk ch
-      // is computed (they read columns 32(ch+1).., the stores of chunk ch write 16ch..16ch+15).
-      // Queries [0, 64) (chunks 0, 1) and [64, 128) (chunks 2, 3) are handed to the MMA warp
-      // separately; dP^T of the second half is read only after its own barrier.
-      uint32_t sbuf[2][32], dbuf[2][32];
-      PA_TMEM_LD32(tA, sbuf[0]);
-      PA_TMEM_LD32(tB, dbuf[0]);
+      // units u = 0..3 of 16 query columns; after units 1 and 3 the 32 packed queries of
+      // the pair are stored (to columns 16(u>>1) ..: the loads in flight then read 32..)
+      uint32_t sb[2][16], db[2][16], pk[16], dk[16];
+      PA_TMEM_LD16(tA, sb[0]);
+      PA_TMEM_LD16(tB, db[0]);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int u = 0; u < 4; ++u) {
         tmem_wait_ld();
-        if (ch == 1) {
-          PA_TMEM_LD32(tA + 64, sbuf[0]);
-        } else if (ch < 3) {
-          PA_TMEM_LD32(tA + 32 * (ch + 1), sbuf[(ch + 1) & 1]);
-          PA_TMEM_LD32(tB + 32 * (ch + 1), dbuf[(ch + 1) & 1]);
+        if (u < 3) {
+          PA_TMEM_LD16(tA + 16 * (u + 1), sb[(u + 1) & 1]);
+          PA_TMEM_LD16(tB + 16 * (u + 1), db[(u + 1) & 1]);
         }
-        const uint32_t (&sv)[32] = sbuf[ch & 1];
-        const uint32_t (&dpv)[32] = dbuf[ch & 1];
-        uint32_t pk[16], dk[16];
+        const uint32_t (&sv)[16] = sb[u & 1];
+        const uint32_t (&dpv)[16] = db[u & 1];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int q = 32 * ch + 2 * k;
+        for (int k = 0; k < 8; ++k) {
+          const int q = 64 * h + 16 * u + 2 * k;
           const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(stage + q);
           const uint64_t nd2 = *reinterpret_cast<const uint64_t*>(stage + 128 + q);
           const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
           const uint64_t pp = ex2x2(x);
           const uint64_t tt = f2_fma(f2_pack(__uint_as_float(dpv[2 * k]), __uint_as_float(dpv[2 * k + 1])), sc2, nd2);
           const uint64_t ds = f2_fma(pp, tt, zero2);
-          pk[k] = key_ok ? pack_bf16x2_pair(pp) : 0u;
-          dk[k] = key_ok ? pack_bf16x2_pair(ds) : 0u;
+          pk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(pp) : 0u;
+          dk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(ds) : 0u;
         }
-        PA_TMEM_ST16(tA + 16 * ch, pk);
-        PA_TMEM_ST16(tB + 16 * ch, dk);
-        // dS^T row t, queries 32ch .. 32ch+31, into the 128-byte-swizzled MN-major layout
-        uint8_t* blk = ds_row + (ch >> 1) * C::kBlockBytes;
+        if (u & 1) {
+          const int ch = u >> 1;
+          PA_TMEM_ST16(tA + 16 * ch, pk);
+          PA_TMEM_ST16(tB + 16 * ch, dk);
+          // dS^T row t, queries 64h + 32ch .. +31, into the 128-byte-swizzled MN-major layout
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = (ch & 1) * 4 + u;
-          *reinterpret_cast<uint4*>(blk + ((c ^ (t & 7)) << 4)) =
-              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        }
-        if (ch & 1) {
-          tmem_wait_st();
-          fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&bars->pds_full[ch >> 1]);
-            if (ch == 3) mbar_arrive(&bars->stage_empty);
-          }
-          if (ch == 1) {
-            ok = mbar_wait(&bars->s_full[1], s_ph, wc);
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-            tc_fence_after();
-            PA_TMEM_LD32(tB + 64, dbuf[0]);
+          for (int v = 0; v < 4; ++v) {
+            const int c = ch * 4 + v;
+            *reinterpret_cast<uint4*>(ds_blk + ((c ^ (t & 7)) << 4)) =
+                make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
           }
         }
       }
-      if (!ok) break;
-      s_ph ^= 1u;
+      tmem_wait_st();
+      fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->pds_full[h]);
+        mbar_arrive(&bars->stage_empty[h]);
+      }
     }
     if (!ok) break;
   }
 }
 
 // ------------------------------------------------------------------ dQ reductions and dK, dV epilogue
+// Warps 12-15: per tile the dQ partial of query row i*128 + t, one column half at a time
+// (each half's columns are released as soon as they are in registers, for the next
+// dP^T half), into the fp32 reductions; at the end of the item dV and dK of key row t.
 template <int D>
 __device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* bars, const WaitCtl& wc, uint32_t tmem) {
   using C = BwdCfg<D>;
   const int t = threadIdx.x & 127;
   const int lane = threadIdx.x & 31;
   const uint32_t lane_base = static_cast<uint32_t>(t & ~31) << 16;
-  const uint32_t tB = tmem + lane_base + C::kColDQ;  // the dQ partial
+  const uint32_t tQ = tmem + lane_base + C::kColDQ;  // the dQ partial
   const uint32_t tDV = tmem + lane_base + C::kColDV;
   const uint32_t tDK = tmem + lane_base + C::kColDK;
   uint32_t sk = 0, dqf_ph = 0, dkvf_ph = 0;
@@ -494,19 +496,22 @@ __device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* ba
       const bool row_ok = qrow < w.len;
       const size_t tok = static_cast<size_t>(w.beg) + qrow;
       float* base = p.dq_acc + (static_cast<size_t>(w.head) * (D / 4) * p.total + tok) * 4;
-      uint32_t o[D];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) PA_TMEM_LD32(tB + 32 * cc, (o + 32 * cc));
-      tmem_wait_ld();
-      // the columns are free as soon as they are in registers
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->dq_empty);
-      if (row_ok) {
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t o[D / 2];
 #pragma unroll
-        for (int u = 0; u < D / 4; ++u)
-          red_add_v4_f32(base + static_cast<size_t>(u) * p.total * 4, __uint_as_float(o[4 * u]),
-                         __uint_as_float(o[4 * u + 1]), __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
+        for (int cc = 0; cc < D / 64; ++cc) PA_TMEM_LD32(tQ + hh * (D / 2) + 32 * cc, (o + 32 * cc));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->dq_empty[hh]);
+        if (row_ok) {
+#pragma unroll
+          for (int u = 0; u < D / 8; ++u)
+            red_add_v4_f32(base + static_cast<size_t>(hh * (D / 8) + u) * p.total * 4, __uint_as_float(o[4 * u]),
+                           __uint_as_float(o[4 * u + 1]), __uint_as_float(o[4 * u + 2]),
+                           __uint_as_float(o[4 * u + 3]));
+        }
       }
     }
     if (!ok) break;
@@ -519,26 +524,21 @@ __device__ __forceinline__ void bwd_reduce_store(const BwdParams& p, BwdBars* ba
     uint4* dvp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dv) + row);
     uint4* dkp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dk) + row);
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t a[32], b[32];
-      PA_TMEM_LD32(tDV + 32 * cc, a);
-      PA_TMEM_LD32(tDK + 32 * cc, b);
+    for (int cc = 0; cc < 2 * (D / 32); ++cc) {
+      const bool is_k = cc >= D / 32;
+      const int c = is_k ? cc - D / 32 : cc;
+      uint32_t a[32];
+      PA_TMEM_LD32((is_k ? tDK : tDV) + 32 * c, a);
       tmem_wait_ld();
+      uint4* dst = is_k ? dkp : dvp;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        uint4 va, vb;
+        uint4 va;
         va.x = pack_bf16x2(__uint_as_float(a[8 * u + 0]), __uint_as_float(a[8 * u + 1]));
         va.y = pack_bf16x2(__uint_as_float(a[8 * u + 2]), __uint_as_float(a[8 * u + 3]));
         va.z = pack_bf16x2(__uint_as_float(a[8 * u + 4]), __uint_as_float(a[8 * u + 5]));
         va.w = pack_bf16x2(__uint_as_float(a[8 * u + 6]), __uint_as_float(a[8 * u + 7]));
-        vb.x = pack_bf16x2(__uint_as_float(b[8 * u + 0]), __uint_as_float(b[8 * u + 1]));
-        vb.y = pack_bf16x2(__uint_as_float(b[8 * u + 2]), __uint_as_float(b[8 * u + 3]));
-        vb.z = pack_bf16x2(__uint_as_float(b[8 * u + 4]), __uint_as_float(b[8 * u + 5]));
-        vb.w = pack_bf16x2(__uint_as_float(b[8 * u + 6]), __uint_as_float(b[8 * u + 7]));
-        if (key_ok) {
-          dvp[cc * 4 + u] = va;
-          dkp[cc * 4 + u] = vb;
-        }
+        if (key_ok) dst[c * 4 + u] = va;
       }
     }
     tc_fence_before();
@@ -562,18 +562,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       mbar_init(&bars->qd_full[s], 1);
       mbar_init(&bars->qd_empty[s], 1);
       mbar_init(&bars->sched_full[s], 1);
-      mbar_init(&bars->sched_empty[s], 9);  // the MMA warp + one lane of each of 8 warps
+      mbar_init(&bars->sched_empty[s], 13);  // the MMA warp + one lane of each of 12 math warps
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&bars->s_full[h], 1);
       mbar_init(&bars->pds_full[h], 4);
     }
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_empty, 4);
     mbar_init(&bars->dkv_full, 1);
     mbar_init(&bars->dkv_empty, 4);
-    mbar_init(&bars->stage_full, 4);
-    mbar_init(&bars->stage_empty, 4);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars->dq_empty[h], 4);
+      mbar_init(&bars->stage_full[h], 4);
+      mbar_init(&bars->stage_empty[h], 4);
+    }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -590,25 +592,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   const int32_t n_items = p.counts[0];
   const int32_t n_sorted = p.counts[1];
   if (warp < 8) {
-    regs_increase<kBwdMathRegs>();
-    if (warp < 4) bwd_elementwise<D>(p, smem, bars, wc, tmem);
-    else bwd_reduce_store<D>(p, bars, wc, tmem);
-    tc_fence_before();
-    named_bar_sync(1, kBwdThreads);
-  } else {
-    regs_decrease<kBwdControlRegs>();
-    if (warp == 8) {
-      if ((threadIdx.x & 31) == 0) bwd_producer<D>(p, smem, bars, wc, n_items, n_sorted);
-    } else if (warp == 9) {
-      bwd_mma<D>(p, smem, bars, wc, tmem);  // the whole warp; one elected lane issues
-    }
-    __syncwarp();
-    tc_fence_before();
-    named_bar_sync(1, kBwdThreads);
-    if (warp == 9) {
-      tc_fence_after();
-      tmem_dealloc(tmem, C::kTmemCols);
-    }
+    bwd_elementwise<D>(p, smem, bars, wc, tmem, warp >> 2);
+  } else if (warp >= 12) {
+    bwd_reduce_store<D>(p, bars, wc, tmem);
+  } else if (warp == 8) {
+    if ((threadIdx.x & 31) == 0) bwd_producer<D>(p, smem, bars, wc, n_items, n_sorted);
+  } else if (warp == 9) {
+    bwd_mma<D>(p, smem, bars, wc, tmem);  // the whole warp; one elected lane issues
+  }
+  __syncwarp();
+  tc_fence_before();
+  named_bar_sync(1, kBwdThreads);
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
