@@ -41,7 +41,16 @@
 
 #include <cstdint>
 
+#include "exp2_poly.cuh"
 #include "sm100_ptx.cuh"
+
+// Key-column pairs of every 4 whose P is exponentiated on the FMA pipe (polynomial,
+// max relative error below 1e-4, far under P's bf16 rounding) instead of the MUFU, in
+// query tiles with no row past the segment end (there every x is finite).
+#ifndef PA_BWD_POLY_PAIRS
+#define PA_BWD_POLY_PAIRS 0
+#endif
+static_assert(PA_BWD_POLY_PAIRS >= 0 && PA_BWD_POLY_PAIRS <= 4, "polynomial share out of range");
 
 namespace pa {
 
@@ -358,6 +367,53 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint8_t* smem, BwdBa
   bwd_drain_wait(&bars->drain, 0, wc.limit_ns);
 }
 
+// P^T and dS^T of one query half: units u = 0..3 of 16 query columns; after units 1
+// and 3 the 32 packed queries of the pair are stored (to columns 16(u>>1) ..: the loads
+// in flight then read 32..).  kPoly of every 4 pairs take the polynomial exponential.
+template <int D, int kPoly>
+__device__ __forceinline__ void bwd_ew_units(uint32_t tA, uint32_t tB, const float* stage, uint8_t* ds_blk, int h,
+                                             int t, bool key_ok, uint64_t c2, uint64_t sc2,
+                                             const Exp2PolyConsts& ek) {
+  const uint64_t zero2 = 0;
+  uint32_t sb[2][16], db[2][16], pk[16], dk[16];
+  PA_TMEM_LD16(tA, sb[0]);
+  PA_TMEM_LD16(tB, db[0]);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    tmem_wait_ld();
+    if (u < 3) {
+      PA_TMEM_LD16(tA + 16 * (u + 1), sb[(u + 1) & 1]);
+      PA_TMEM_LD16(tB + 16 * (u + 1), db[(u + 1) & 1]);
+    }
+    const uint32_t (&sv)[16] = sb[u & 1];
+    const uint32_t (&dpv)[16] = db[u & 1];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int q = 64 * h + 16 * u + 2 * k;
+      const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(stage + q);
+      const uint64_t nd2 = *reinterpret_cast<const uint64_t*>(stage + 128 + q);
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
+      const uint64_t pp = (k & 3) >= 4 - kPoly ? ex2x2_poly(x, ek) : ex2x2(x);
+      const uint64_t tt = f2_fma(f2_pack(__uint_as_float(dpv[2 * k]), __uint_as_float(dpv[2 * k + 1])), sc2, nd2);
+      const uint64_t ds = f2_fma(pp, tt, zero2);
+      pk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(pp) : 0u;
+      dk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(ds) : 0u;
+    }
+    if (u & 1) {
+      const int ch = u >> 1;
+      PA_TMEM_ST16(tA + 16 * ch, pk);
+      PA_TMEM_ST16(tB + 16 * ch, dk);
+      // dS^T row t, queries 64h + 32ch .. +31, into the 128-byte-swizzled MN-major layout
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int c = ch * 4 + v;
+        *reinterpret_cast<uint4*>(ds_blk + ((c ^ (t & 7)) << 4)) =
+            make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ elementwise: P^T, dS^T
 // Warpgroup h (warps 4h .. 4h+3) computes P^T and dS^T of queries [64h, 64h + 64) of
 // every tile, one thread per key row, in units of 16 query columns (the loads of unit
@@ -376,7 +432,9 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
   uint8_t* ds_blk = smem + C::kOffDS + h * C::kBlockBytes + t * 128;
   const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
   const uint64_t sc2 = f2_pack(p.scale, p.scale);
-  const uint64_t zero2 = 0;
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  const Exp2PolyConsts ek{f2_pack(magic, magic), f2_pack(-magic, -magic), f2_pack(kExp2C0, kExp2C0),
+                          f2_pack(kExp2C1, kExp2C1), f2_pack(kExp2C2, kExp2C2), f2_pack(kExp2C3, kExp2C3)};
   uint32_t sk = 0, s_ph = 0, st_ph = 0;
   for (;;) {
     BwdItem w;
@@ -413,45 +471,10 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint8_t* sme
       if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
       s_ph ^= 1u;
       tc_fence_after();
-      // units u = 0..3 of 16 query columns; after units 1 and 3 the 32 packed queries of
-      // the pair are stored (to columns 16(u>>1) ..: the loads in flight then read 32..)
-      uint32_t sb[2][16], db[2][16], pk[16], dk[16];
-      PA_TMEM_LD16(tA, sb[0]);
-      PA_TMEM_LD16(tB, db[0]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        tmem_wait_ld();
-        if (u < 3) {
-          PA_TMEM_LD16(tA + 16 * (u + 1), sb[(u + 1) & 1]);
-          PA_TMEM_LD16(tB + 16 * (u + 1), db[(u + 1) & 1]);
-        }
-        const uint32_t (&sv)[16] = sb[u & 1];
-        const uint32_t (&dpv)[16] = db[u & 1];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int q = 64 * h + 16 * u + 2 * k;
-          const uint64_t nl2 = *reinterpret_cast<const uint64_t*>(stage + q);
-          const uint64_t nd2 = *reinterpret_cast<const uint64_t*>(stage + 128 + q);
-          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
-          const uint64_t pp = ex2x2(x);
-          const uint64_t tt = f2_fma(f2_pack(__uint_as_float(dpv[2 * k]), __uint_as_float(dpv[2 * k + 1])), sc2, nd2);
-          const uint64_t ds = f2_fma(pp, tt, zero2);
-          pk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(pp) : 0u;
-          dk[8 * (u & 1) + k] = key_ok ? pack_bf16x2_pair(ds) : 0u;
-        }
-        if (u & 1) {
-          const int ch = u >> 1;
-          PA_TMEM_ST16(tA + 16 * ch, pk);
-          PA_TMEM_ST16(tB + 16 * ch, dk);
-          // dS^T row t, queries 64h + 32ch .. +31, into the 128-byte-swizzled MN-major layout
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int c = ch * 4 + v;
-            *reinterpret_cast<uint4*>(ds_blk + ((c ^ (t & 7)) << 4)) =
-                make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
-          }
-        }
-      }
+      if (PA_BWD_POLY_PAIRS > 0 && (i + 1) * 128 <= w.len)
+        bwd_ew_units<D, PA_BWD_POLY_PAIRS>(tA, tB, stage, ds_blk, h, t, key_ok, c2, sc2, ek);
+      else
+        bwd_ew_units<D, 0>(tA, tB, stage, ds_blk, h, t, key_ok, c2, sc2, ek);
       tmem_wait_st();
       fence_proxy_async_smem();  // the dS^T stores are read by the tensor core
       tc_fence_before();
