@@ -282,6 +282,40 @@ def kernel_ms(pa, call, flush, steps, flush_each=True):
     return tot / max(1, n), dt
 
 
+def paired_steps(pa, call, flush, stream, warmup, steps, world, device):
+    """Per-call times and the main kernel's time from one region: `steps` pairs of calls, L2
+    flushed before each; the first call of a pair is bracketed by CUDA events, the second runs
+    with the library's kernel events on. Both numbers then come from the same clock and power
+    state (two back-to-back loops can see different ones). Returns (per-call ms list, kernel
+    ms average)."""
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    pa.pa_profile_read()  # clear
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.fill_(1.0)
+        a.record(stream)
+        call()
+        b.record(stream)
+        flush.fill_(1.0)
+        pa.pa_profile_enable(True)
+        call()
+        pa.pa_profile_enable(False)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor(ms, dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.tolist()
+    tot, n = pa.pa_profile_read()
+    return ms, tot / max(1, n)
+
+
 def unique_bytes(T, H, d):
     """Algorithmic HBM bytes of one forward call: q, k, v read and out written (bf16), lse written (fp32)."""
     return 4.0 * T * H * d * 2 + 4.0 * T * H
@@ -321,8 +355,7 @@ def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5):
     torch.cuda.synchronize()
     est = max(time.time() - t0, 1e-5)
     steps = max(5, min(args.steps, int(target_s / est)))
-    ms, _, _ = time_steps(pack, flush, stream, args.warmup, steps, world, device)
-    kms, _ = kernel_ms(pa, pack, flush, steps)
+    ms, kms = paired_steps(pa, pack, flush, stream, args.warmup, steps, world, device)
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, pack.cfg["name"])
@@ -398,31 +431,8 @@ def run_ours(args, world, rank, local):
         if rc != pa.PA_OK:
             raise pa.PackAttnError(rc, "pa_varlen_attn_bwd")
 
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        bwd_call()
-    torch.cuda.synchronize()
-    bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.fill_(1.0)
-        bev[i][0].record(stream)
-        bwd_call()
-        bev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    bwd_step_ms = [a.elapsed_time(b) for a, b in bev]
-    pa.pa_profile_read()  # clear
-    pa.pa_profile_enable(True)
-    t_bprof0 = time.time()
-    for i in range(args.steps):
-        flush.fill_(1.0)
-        bwd_call()
-    torch.cuda.synchronize()
-    t_bprof = time.time() - t_bprof0
-    pa.pa_profile_enable(False)
-    bkern_ms_total, bkern_n = pa.pa_profile_read()
+    bwd_step_ms, bkern_ms = paired_steps(pa, bwd_call, flush, stream, args.warmup, args.steps, world, device)
+    t_bprof = 2e-3 * sum(bwd_step_ms)  # the paired region's length, about
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, "backward region")
@@ -687,9 +697,9 @@ def run_ours(args, world, rank, local):
             "value": bwd_flops * world / (bwd_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": bwd_ms,
             "step_ms_p10_p50_p90": [bq10, bq50, bq90], "valid_flops_per_step": bwd_flops,
             "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel<%d>" % d,
-                         "achieved": bwd_flops / (bkern_ms_total / max(1, bkern_n) * 1e-3) / 1e12,
+                         "achieved": bwd_flops / (bkern_ms * 1e-3) / 1e12,
                          "peak": bpeak, "unit": "TFLOP/s",
-                         "frac": bwd_flops / (bkern_ms_total / max(1, bkern_n) * 1e-3) / 1e12 / bpeak,
+                         "frac": bwd_flops / (bkern_ms * 1e-3) / 1e12 / bpeak,
                          "peak_source": bpeak_src, "traffic": None},
             "gpu_launches": 4 * args.steps,  # prep, schedule, main, dq conversion per step
         },
