@@ -218,10 +218,10 @@ def run_reference(args, world, rank):
 HEADLINE_METRIC = "varlen attn fwd effective TFLOP/s (valid FLOPs) on 1 B200; % of BF16 peak"
 
 
-def traffic_for_current_kernel():
-    """DRAM bytes per launch from the committed ncu summary, if it matches the kernel source as built."""
+def traffic_for_current_kernel(record="attn_fwd_traffic.json"):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the kernel source as built."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    path = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -616,6 +616,7 @@ def run_ours(args, world, rank, local):
     bpeak_src = (f"bf16_tflops_sustained ({peak_src}; kernel timed inside {t_bprof:.2f} s of back-to-back steps)"
                  if t_bprof >= 0.25 else f"bf16_tflops ({peak_src}, burst)")
     trec = traffic_for_current_kernel()
+    btrec = traffic_for_current_kernel("attn_bwd_traffic.json")
     ss_achieved = flops / (ss_kern_ms * 1e-3) / 1e12
     steady = {
         "what": (f"{n_ss} back-to-back calls of the same pack, no idle gap and no L2 flush between them "
@@ -700,7 +701,9 @@ def run_ours(args, world, rank, local):
                          "achieved": bwd_flops / (bkern_ms * 1e-3) / 1e12,
                          "peak": bpeak, "unit": "TFLOP/s",
                          "frac": bwd_flops / (bkern_ms * 1e-3) / 1e12 / bpeak,
-                         "peak_source": bpeak_src, "traffic": None},
+                         "peak_source": bpeak_src,
+                         "traffic": (btrec or {}).get("dram_bytes_per_launch"),
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
             "gpu_launches": 4 * args.steps,  # prep, schedule, main, dq conversion per step
         },
         "projections": {
