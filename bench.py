@@ -316,6 +316,53 @@ def paired_steps(pa, call, flush, stream, warmup, steps, world, device):
     return ms, tot / max(1, n)
 
 
+def fp8_compare(pa, pack, flush, stream, warmup, steps):
+    """bf16 call against the FP8 path on one pack (d = 128), interleaved step by step so that
+    all four see the same clocks: the bf16 call; the quantiser (maxima of this call) + FP8
+    attention; the delayed-scaling quantiser (a previous step's maxima) + FP8 attention; the FP8
+    attention alone. L2 flushed before each; returns the mean ms of each."""
+    T, H, d = pack.T, pack.H, pack.d
+    dev = pack.q.device
+    B = pack.cu.numel() - 1
+    q8, k8 = (torch.empty(T, H, d, dtype=torch.uint8, device=dev) for _ in range(2))
+    v8t = torch.empty(H * d, pa.pa_fp8_vt_keys(B, T), dtype=torch.uint8, device=dev)
+    sc8 = torch.empty(4 + H * d, dtype=torch.float32, device=dev)
+    out8, lse8 = torch.empty_like(pack.out), torch.empty_like(pack.lse)
+    am_in = torch.ones(4 + H * d, dtype=torch.float32, device=dev)
+    am_out = torch.empty_like(am_in)
+
+    def check(rc, what):
+        if rc != pa.PA_OK:
+            raise pa.PackAttnError(rc, what)
+
+    check(pa.pa_fp8_quantize_qkv_delayed(pack.q, pack.k, pack.v, pack.cu, am_out, am_in, q8, k8, v8t, sc8, stream),
+          "pa_fp8_quantize_qkv_delayed")  # am_in = this pack's maxima (a previous step's record)
+    quant = lambda: check(pa.pa_fp8_quantize_qkv(pack.q, pack.k, pack.v, pack.cu, q8, k8, v8t, sc8, stream),
+                          "pa_fp8_quantize_qkv")
+    dquant = lambda: check(pa.pa_fp8_quantize_qkv_delayed(pack.q, pack.k, pack.v, pack.cu, am_in, am_out, q8, k8,
+                                                          v8t, sc8, stream), "pa_fp8_quantize_qkv_delayed")
+    attn = lambda: check(pa.pa_varlen_attn_fwd_fp8(q8, k8, v8t, sc8, pack.cu, pack.p["max_seqlen"],
+                                                   pack.p["scale"], out8, lse8, stream), "pa_varlen_attn_fwd_fp8")
+    arms = [pack, lambda: (quant(), attn()), lambda: (dquant(), attn()), attn]
+    for _ in range(warmup):
+        for fn in arms:
+            flush.fill_(1.0)
+            fn()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in arms]
+          for _ in range(steps)]
+    for row in ev:
+        for fn, (a, b) in zip(arms, row):
+            flush.fill_(1.0)
+            a.record(stream)
+            fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    check(pa.pa_get_error(stream), "fp8 comparison")
+    ms = [sum(row[i][0].elapsed_time(row[i][1]) for row in ev) / steps for i in range(len(arms))]
+    return dict(bf16_ms=ms[0], quant_attn_ms=ms[1], delayed_attn_ms=ms[2], attn_ms=ms[3], steps=steps)
+
+
 def unique_bytes(T, H, d):
     """Algorithmic HBM bytes of one forward call: q, k, v read and out written (bf16), lse written (fp32)."""
     return 4.0 * T * H * d * 2 + 4.0 * T * H
@@ -494,9 +541,24 @@ def run_ours(args, world, rank, local):
             if rc != pa.PA_OK:
                 raise pa.PackAttnError(rc, "pa_varlen_attn_fwd_fp8")
 
+        # delayed scaling: one pass with the maxima of a previous step (here the same tensors'
+        # maxima, recorded by a first call), this call's maxima returned for the next step
+        am_prev = torch.ones(4 + H * d, dtype=torch.float32, device=device)
+        am_in, am_out = torch.empty_like(am_prev), torch.empty_like(am_prev)
+        if pa.pa_fp8_quantize_qkv_delayed(q, k, v, cu, am_prev, am_in, q8, k8, v8t, sc8, stream) != pa.PA_OK:
+            raise RuntimeError("pa_fp8_quantize_qkv_delayed")
+
+        def dquant_call():
+            rc = pa.pa_fp8_quantize_qkv_delayed(q, k, v, cu, am_in, am_out, q8, k8, v8t, sc8, stream)
+            if rc != pa.PA_OK:
+                raise pa.PackAttnError(rc, "pa_fp8_quantize_qkv_delayed")
+
         quant_ms = proj_time(quant_call)
+        dquant_ms = proj_time(dquant_call)
         fp8_ms = proj_time(fp8_call)
         both_ms = proj_time(lambda: (quant_call(), fp8_call()))
+        dboth_ms = proj_time(lambda: (dquant_call(), fp8_call()))
+        bf16_ms = proj_time(call)  # the bf16 call again, in the same stretch of the run
         pa.pa_profile_read()  # clear
         pa.pa_profile_enable(True)
         t_fprof0 = time.time()
@@ -511,6 +573,7 @@ def run_ours(args, world, rank, local):
         if rc != pa.PA_OK:
             raise pa.PackAttnError(rc, "fp8 region")
         fp8_rec = dict(quant_ms=quant_ms, fp8_ms=fp8_ms, both_ms=both_ms, t_prof=t_fprof,
+                       dquant_ms=dquant_ms, dboth_ms=dboth_ms, bf16_ms=bf16_ms,
                        kern_s=fkern_ms_total / max(1, fkern_n) * 1e-3,
                        # algorithmic bytes: q, k, v read once (6 B per element) and the E4M3 codes
                        # written (3 B); the two-pass quantiser moves 15 B (the amax pass reads
@@ -586,6 +649,8 @@ def run_ours(args, world, rank, local):
             rec = measure_pack(pa, pk, flush, stream, args, world, device)
             rec.update(tokens=pk.T, segments=len(pk.segs), heads=pk.H, head_dim=pk.d, valid_flops=pk.flops,
                        unique_bytes=pk.bytes)
+            if pk.d == 128 and name in workloads.CONFIG_NAMES and name != "tiny":
+                rec["fp8"] = fp8_compare(pa, pk, flush, stream, args.warmup, rec["steps"])
             if name in workloads.SHORT_PACK_NAMES or name == "tiny":
                 # the same pack with short-segment packing off: every segment its own tiles
                 pa.pa_set_short_packing(False)
@@ -646,6 +711,15 @@ def run_ours(args, world, rank, local):
              "kernel": {"name": head_kernel_name(rec["head_dim"]), "ms": rec["kernel_ms"],
                         "achieved": rec["kernel_tflops"], "frac": rec["kernel_tflops"] / peak_burst,
                         "peak": peak_burst, "peak_source": f"bf16_tflops ({peak_src}, burst)"}}
+        f8 = rec.get("fp8")
+        if f8:
+            r["fp8_vs_bf16"] = {
+                "what": "per call, interleaved step by step with the bf16 call (same clocks), L2 flushed",
+                "bf16_ms": f8["bf16_ms"], "fp8_attention_ms": f8["attn_ms"],
+                "quantiser_plus_attention_ms": f8["quant_attn_ms"],
+                "delayed_quantiser_plus_attention_ms": f8["delayed_attn_ms"],
+                "speedup_quantiser_plus_attention": f8["bf16_ms"] / f8["quant_attn_ms"],
+                "speedup_delayed_quantiser_plus_attention": f8["bf16_ms"] / f8["delayed_attn_ms"]}
         if name in workloads.SHORT_PACK_NAMES or name == "tiny":
             # short-segment regime: bound by HBM (per-segment intensity about L/2 FLOP per byte, below
             # the ridge of about 259 FLOP/B for L < ~520); unique bytes / time
@@ -730,6 +804,20 @@ def run_ours(args, world, rank, local):
                                        "kernels": "memset + fp8_amax_kernel + fp8_quantize_kernel"}},
             "quantiser_plus_attention": {"value": flops * world / (fp8_rec["both_ms"] * 1e-3) / 1e12,
                                          "unit": "TFLOP/s", "ms_per_step": fp8_rec["both_ms"]},
+            "delayed_quantiser": {"ms_per_step": fp8_rec["dquant_ms"], "launches_per_step": 2,
+                                  "note": "one pass: scales from a previous step's maxima, this call's maxima "
+                                          "returned (pa_fp8_quantize_qkv_delayed)",
+                                  "roofline": {"bound": "hbm", "unit": "GB/s", "bytes_per_call": fp8_rec["quant_bytes"],
+                                               "achieved": fp8_rec["quant_bytes"] / (fp8_rec["dquant_ms"] * 1e-3) / 1e9,
+                                               "peak": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                               "frac": fp8_rec["quant_bytes"] / (fp8_rec["dquant_ms"] * 1e-3) / 1e9 /
+                                               float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                               "kernels": "memset of amax_out + fp8_quantize_kernel<true>"}},
+            "delayed_quantiser_plus_attention": {"value": flops * world / (fp8_rec["dboth_ms"] * 1e-3) / 1e12,
+                                                 "unit": "TFLOP/s", "ms_per_step": fp8_rec["dboth_ms"]},
+            "bf16_same_stretch": {"value": flops * world / (fp8_rec["bf16_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                  "ms_per_step": fp8_rec["bf16_ms"],
+                                  "note": "the bf16 call timed again next to the FP8 timings (same clocks)"},
             "roofline": {"bound": "tensor", "kernel": "attn_fwd_fp8_kernel",
                          "achieved": flops / fp8_rec["kern_s"] / 1e12,
                          "peak": 2.0 * (float(peaks.get("bf16_tflops_sustained",

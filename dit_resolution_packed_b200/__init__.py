@@ -68,6 +68,8 @@ def load_library(path=None):
     lib.pa_fp8_vt_keys.argtypes = [i32, i32]
     lib.pa_fp8_quantize_qkv.restype = ctypes.c_int
     lib.pa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+    lib.pa_fp8_quantize_qkv_delayed.restype = ctypes.c_int
+    lib.pa_fp8_quantize_qkv_delayed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.pa_varlen_attn_fwd_fp8.restype = ctypes.c_int
     lib.pa_varlen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp]
     lib.pa_get_error.restype = ctypes.c_int
@@ -309,6 +311,45 @@ def fp8_quantize_qkv(q, k, v, cu_seqlens, stream=None):
     rc = pa_fp8_quantize_qkv(q, k, v, cu_seqlens, qz["q8"], qz["k8"], qz["v8t"], qz["scales"], stream)
     if rc != PA_OK:
         raise PackAttnError(rc, "pa_fp8_quantize_qkv")
+    return qz
+
+
+def pa_fp8_quantize_qkv_delayed(q, k, v, cu_seqlens, amax_in, amax_out, q8, k8, v8t, scales, stream=None):
+    """C ``pa_fp8_quantize_qkv_delayed``: as ``pa_fp8_quantize_qkv`` with the scales from amax_in (fp32
+    [4 + H*128]); this call's maxima go to amax_out (same layout).  Returns the status code."""
+    import torch
+    _check_bf16(q=q, k=k, v=v)
+    _check_bytes(q8=q8, k8=k8, v8t=v8t)
+    for name, t in (("scales", scales), ("amax_in", amax_in), ("amax_out", amax_out)):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous float32 tensor")
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    if (k.shape != q.shape or v.shape != q.shape or q8.shape != q.shape or k8.shape != q.shape
+            or tuple(v8t.shape) != (H * d, pa_fp8_vt_keys(B, T)) or scales.numel() != 4 + H * d
+            or amax_in.numel() != 4 + H * d or amax_out.numel() != 4 + H * d):
+        raise ValueError("shape mismatch: q, k, v, q8, k8 [T, H, d]; v8t [H*d, keys]; scales, amax [4 + H*d]")
+    return load_library().pa_fp8_quantize_qkv_delayed(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), B, T, H, d, _ptr(amax_in), _ptr(amax_out), _ptr(q8), _ptr(k8),
+        _ptr(v8t), _ptr(scales), _stream_handle(stream))
+
+
+def fp8_quantize_qkv_delayed(q, k, v, cu_seqlens, amax_in, stream=None):
+    """Delayed-scaling quantiser: scales from amax_in; returns the dict of ``fp8_quantize_qkv`` plus
+    ``amax`` (this call's maxima, fp32 [4 + H*128], for the next call)."""
+    import torch
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    dev = q.device
+    qz = dict(q8=torch.empty(T, H, d, dtype=torch.uint8, device=dev),
+              k8=torch.empty(T, H, d, dtype=torch.uint8, device=dev),
+              v8t=torch.empty(H * d, max(pa_fp8_vt_keys(B, T), 0), dtype=torch.uint8, device=dev),
+              scales=torch.empty(4 + H * d, dtype=torch.float32, device=dev),
+              amax=torch.empty(4 + H * d, dtype=torch.float32, device=dev))
+    rc = pa_fp8_quantize_qkv_delayed(q, k, v, cu_seqlens, amax_in, qz["amax"], qz["q8"], qz["k8"], qz["v8t"],
+                                     qz["scales"], stream)
+    if rc != PA_OK:
+        raise PackAttnError(rc, "pa_fp8_quantize_qkv_delayed")
     return qz
 
 

@@ -606,17 +606,22 @@ __device__ __forceinline__ uint2 quant8(uint4 x, float m) {
 // [h * 128 + c][key] with segment s's keys starting at 16*ceil(cu[s]/16) + 16*s
 // (for token t of segment s: key t + 16*ceil(cu[s]/16) + 16*s - cu[s]).
 // Also writes the scales: [0] s_q, [1] s_k, [4 + h * 128 + c] s_v.
+// kTrack: the maxima of this call's q, k, v are also accumulated into amax_out (same
+// layout as amax, zeroed by the caller), for the next call's scales (delayed scaling).
+template <bool kTrack>
 __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
     const uint4* q, const uint4* k, const uint4* v, const int32_t* cu, int32_t batch, int32_t total, int32_t heads,
-    const uint32_t* amax, uint2* q8, uint2* k8, uint8_t* v8t, int64_t vt_keys, float* scales) {
+    const uint32_t* amax, uint2* q8, uint2* k8, uint8_t* v8t, int64_t vt_keys, float* scales, uint32_t* amax_out) {
   constexpr int D = 128;
   __shared__ __align__(16) uint8_t s_t[D][128 + 4];  // [channel][token] of this tile (word-aligned rows)
   __shared__ float s_mv[D];
   __shared__ int64_t s_off[128];
   __shared__ int s_vec[8];  // 16-token chunk goes out as one 16-byte store
+  __shared__ uint32_t s_am[kTrack ? D + 2 : 1];  // this tile's maxima: v per channel, then q, k
   const int h = blockIdx.x;
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * 128;
   const float mq = fp8_mult(__ldg(amax)), mk = fp8_mult(__ldg(amax + 1));
+  if (kTrack && threadIdx.x < D + 2) s_am[threadIdx.x] = 0u;
   if (threadIdx.x < D) {
     const uint32_t a = __ldg(amax + 4 + h * D + threadIdx.x);
     s_mv[threadIdx.x] = fp8_mult(a);
@@ -646,18 +651,29 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
   __syncthreads();
   // q, k: 8 codes per 16-byte load; v: four tokens of one 8-channel chunk per thread, so
   // that each channel's four codes go to the transposed tile as one 32-bit word
+  uint32_t tq = 0u, tk = 0u;  // pairs of bf16 magnitudes (kTrack)
   for (int i = threadIdx.x; i < 32 * (D / 8); i += kQuantThreads) {
     const int tg = i >> 4, c8 = i & 15;
     uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // [channel of the chunk]: 4 token bytes
+    uint32_t tv[4] = {0u, 0u, 0u, 0u};                   // pairs of bf16 magnitudes of v (kTrack)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int64_t t = t0 + tg * 4 + u;
       if (t >= total) break;
       const int64_t idx = (t * heads + h) * (D / 8) + c8;
-      q8[idx] = quant8(__ldg(q + idx), mq);
-      k8[idx] = quant8(__ldg(k + idx), mk);
+      const uint4 a = __ldg(q + idx), b = __ldg(k + idx);
+      q8[idx] = quant8(a, mq);
+      k8[idx] = quant8(b, mk);
       const uint4 x = __ldg(v + idx);
       const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      if (kTrack) {
+        tq = __vmaxu2(tq, __vmaxu2(__vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu),
+                                   __vmaxu2(a.z & 0x7FFF7FFFu, a.w & 0x7FFF7FFFu)));
+        tk = __vmaxu2(tk, __vmaxu2(__vmaxu2(b.x & 0x7FFF7FFFu, b.y & 0x7FFF7FFFu),
+                                   __vmaxu2(b.z & 0x7FFF7FFFu, b.w & 0x7FFF7FFFu)));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tv[e] = __vmaxu2(tv[e], w[e] & 0x7FFF7FFFu);
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int c = c8 * 8 + 2 * e;
@@ -670,8 +686,34 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) *reinterpret_cast<uint32_t*>(&s_t[c8 * 8 + e][tg * 4]) = pk[e];
+    if (kTrack) {  // bf16 magnitude bits << 16 are the fp32 bits of the same value
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (tv[e] & 0xFFFFu) atomicMax(&s_am[c8 * 8 + 2 * e], (tv[e] & 0xFFFFu) << 16);
+        if (tv[e] >> 16) atomicMax(&s_am[c8 * 8 + 2 * e + 1], (tv[e] >> 16) << 16);
+      }
+    }
+  }
+  if (kTrack) {
+    uint32_t fq = max(tq & 0xFFFFu, tq >> 16) << 16, fk = max(tk & 0xFFFFu, tk >> 16) << 16;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      fq = max(fq, __shfl_xor_sync(0xffffffffu, fq, o));
+      fk = max(fk, __shfl_xor_sync(0xffffffffu, fk, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      if (fq) atomicMax(&s_am[D], fq);
+      if (fk) atomicMax(&s_am[D + 1], fk);
+    }
   }
   __syncthreads();
+  if (kTrack) {
+    if (threadIdx.x < D) {
+      if (s_am[threadIdx.x]) atomicMax(amax_out + 4 + h * D + threadIdx.x, s_am[threadIdx.x]);
+    } else if (threadIdx.x < D + 2) {
+      if (s_am[threadIdx.x]) atomicMax(amax_out + threadIdx.x - D, s_am[threadIdx.x]);
+    }
+  }
   // v8^T rows, one warp per channel row: a 16-token chunk goes out as one 16-byte store
   // when its tokens lie in one segment (equal key offsets: the offset grows at every
   // segment start) and its first key is 16-byte aligned (decided once per block, the

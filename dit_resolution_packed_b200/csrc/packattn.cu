@@ -849,13 +849,35 @@ int64_t pa_fp8_vt_keys(int32_t batch, int32_t total_tokens) {
   return fp8_vt_keys(batch, total_tokens);
 }
 
-int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
-                        int32_t total_tokens, int32_t heads, int32_t head_dim, void* q8, void* k8, void* v8t,
-                        float* scales, void* stream_handle) {
+namespace {
+// The FP8 quantiser. amax_in null: the maxima of this call's q, k, v (a first pass)
+// give the scales. Otherwise amax_in's maxima do (delayed scaling: one pass), and this
+// call's maxima go to amax_out.
+int fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                 int32_t total_tokens, int32_t heads, int32_t head_dim, const float* amax_in, float* amax_out,
+                 void* q8, void* k8, void* v8t, float* scales, void* stream_handle) {
   if (head_dim != 128) return PA_ERR_HEAD_DIM;
   if (heads < 1 || batch < 0 || total_tokens < 0) return PA_ERR_SHAPE;
   if (batch == 0 && total_tokens > 0) return PA_ERR_SHAPE;
-  if (batch == 0 || total_tokens == 0) return PA_OK;
+  const bool delayed = amax_in != nullptr || amax_out != nullptr;
+  if (delayed && (!amax_in || !amax_out)) return PA_ERR_NULL;
+  const size_t amax_bytes = 4 * (4 + static_cast<size_t>(heads) * head_dim);
+  if (delayed) {
+    if (!aligned(amax_in, 4) || !aligned(amax_out, 4)) return PA_ERR_ALIGN;
+    const uintptr_t ai = reinterpret_cast<uintptr_t>(amax_in), ao = reinterpret_cast<uintptr_t>(amax_out);
+    if (ai < ao + amax_bytes && ao < ai + amax_bytes) return PA_ERR_SHAPE;  // the two must not overlap
+  }
+  if (batch == 0 || total_tokens == 0) {
+    if (!delayed) return PA_OK;
+    // no tokens: this call's maxima are all zero
+    int dev0 = -1, rc0;
+    if ((rc0 = device_of(amax_out, &dev0)) != PA_OK) return rc0;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (cudaSetDevice(dev0) != cudaSuccess) return PA_ERR_CUDA;
+    return cudaMemsetAsync(amax_out, 0, amax_bytes, static_cast<cudaStream_t>(stream_handle)) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+  }
   if (!q || !k || !v || !cu_seqlens || !q8 || !k8 || !v8t || !scales) return PA_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) || !aligned(k8, 16) ||
       !aligned(v8t, 16) || !aligned(scales, 16) || !aligned(cu_seqlens, 4))
@@ -867,7 +889,7 @@ int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32
   int dev = -1, d2 = -1;
   int rc;
   if ((rc = device_of(q, &dev)) != PA_OK) return rc;
-  const void* others[7] = {k, v, cu_seqlens, q8, k8, v8t, scales};
+  const void* others[9] = {k, v, cu_seqlens, q8, k8, v8t, scales, delayed ? amax_in : q, delayed ? amax_out : q};
   for (const void* p : others) {
     if ((rc = device_of(p, &d2)) != PA_OK) return rc;
     if (d2 != dev) return PA_ERR_NOT_DEVICE;
@@ -876,9 +898,18 @@ int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32
   std::lock_guard<std::mutex> lock(g_mu);
   if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
   if ((rc = ensure_device(dev)) != PA_OK) return rc;
+  const dim3 qgrid(heads, static_cast<unsigned>(tiles));
+  const int64_t vt_keys = fp8_vt_keys(batch, total_tokens);
+  if (delayed) {
+    if (cudaMemsetAsync(amax_out, 0, amax_bytes, stream) != cudaSuccess) return PA_ERR_CUDA;
+    pa::fp8_quantize_kernel<true><<<qgrid, pa::kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, batch,
+        total_tokens, heads, reinterpret_cast<const uint32_t*>(amax_in), static_cast<uint2*>(q8),
+        static_cast<uint2*>(k8), static_cast<uint8_t*>(v8t), vt_keys, scales, reinterpret_cast<uint32_t*>(amax_out));
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
   StreamState* st = state_for(dev, stream);
   if ((rc = ensure_status(st)) != PA_OK) return rc;
-  const size_t amax_bytes = 4 * (4 + static_cast<size_t>(heads) * head_dim);
   if ((rc = ensure_workspace(st, amax_bytes)) != PA_OK) return rc;
   uint32_t* amax = reinterpret_cast<uint32_t*>(st->ws);
   if (cudaMemsetAsync(amax, 0, amax_bytes, stream) != cudaSuccess) return PA_ERR_CUDA;
@@ -890,11 +921,28 @@ int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), total_tokens, nch8,
       amax);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  pa::fp8_quantize_kernel<<<dim3(heads, static_cast<unsigned>(tiles)), pa::kQuantThreads, 0, stream>>>(
+  pa::fp8_quantize_kernel<false><<<qgrid, pa::kQuantThreads, 0, stream>>>(
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, batch,
       total_tokens, heads, amax, static_cast<uint2*>(q8), static_cast<uint2*>(k8), static_cast<uint8_t*>(v8t),
-      fp8_vt_keys(batch, total_tokens), scales);
+      vt_keys, scales, nullptr);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+}  // namespace
+
+int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                        int32_t total_tokens, int32_t heads, int32_t head_dim, void* q8, void* k8, void* v8t,
+                        float* scales, void* stream_handle) {
+  return fp8_quantize(q, k, v, cu_seqlens, batch, total_tokens, heads, head_dim, nullptr, nullptr, q8, k8, v8t,
+                      scales, stream_handle);
+}
+
+int pa_fp8_quantize_qkv_delayed(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                const float* amax_in, float* amax_out, void* q8, void* k8, void* v8t, float* scales,
+                                void* stream_handle) {
+  if (!amax_in || !amax_out) return PA_ERR_NULL;
+  return fp8_quantize(q, k, v, cu_seqlens, batch, total_tokens, heads, head_dim, amax_in, amax_out, q8, k8, v8t,
+                      scales, stream_handle);
 }
 
 int pa_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8t, const float* scales,

@@ -197,6 +197,29 @@ PA_API int pa_fp8_quantize_qkv(const void* q, const void* k, const void* v, cons
                                void* k8, void* v8t, float* scales, void* stream);
 
 /*
+ * pa_fp8_quantize_qkv_delayed -- the same quantisation in one pass over q, k, v, with
+ * the scales taken from given maxima instead of this call's (delayed scaling: the
+ * maxima of the previous step of a training or serving loop; the pages fix the
+ * granularity -- q, k per tensor, v per channel -- not where the maxima come from).
+ *   amax_in      device, fp32, [4 + heads*128], 4-byte aligned (read): a_q at [0],
+ *                a_k at [1], a of v's column (h, c) at [4 + h*128 + c]; finite and
+ *                non-negative (as amax_out holds them).  mult, s and code follow from
+ *                these a exactly as in pa_fp8_quantize_qkv; an input above its a is
+ *                clamped to the code of +-448.
+ *   amax_out     device, fp32, [4 + heads*128], 4-byte aligned (written): the absolute
+ *                maxima of this call's q, k and v columns, in amax_in's layout (exact:
+ *                the largest |bf16| of each group, widened), for the next call.  Must
+ *                not overlap amax_in (PA_ERR_SHAPE).
+ * Other arguments as for pa_fp8_quantize_qkv.  Workspace: none.  With batch = 0 or
+ * total_tokens = 0, amax_out is zeroed and nothing else is written.  Errors:
+ * PA_ERR_NULL for a null amax_in or amax_out; otherwise as pa_fp8_quantize_qkv.
+ */
+PA_API int pa_fp8_quantize_qkv_delayed(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                       int32_t batch, int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                       const float* amax_in, float* amax_out, void* q8, void* k8, void* v8t,
+                                       float* scales, void* stream);
+
+/*
  * pa_varlen_attn_fwd_fp8 -- the packed varlen attention forward on the quantiser's
  * output (q8, k8, v8t, scales as pa_fp8_quantize_qkv writes them; the same pack,
  * heads and cu_seqlens).  Computes, with x = scale * s_q * s_k * (q8 . k8) per key,

@@ -107,21 +107,37 @@ def quantize(x, amax):
     return out.reshape(prod.shape)
 
 
+def qkv_amax(q, k, v):
+    """(a_q, a_k, a_v): the absolute maxima of the whole q, the whole k and each (head,
+    channel) column of v over all tokens (fp32; zero for an empty tensor)."""
+    qf, kf, vf = _f32(q), _f32(k), _f32(v)
+    aq = np.float32(np.max(np.abs(qf))) if qf.size else np.float32(0)
+    ak = np.float32(np.max(np.abs(kf))) if kf.size else np.float32(0)
+    av = (np.max(np.abs(vf), axis=0) if vf.shape[0] else np.zeros(vf.shape[1:])).astype(np.float32)
+    return aq, ak, av
+
+
+def quantize_qkv_with(q, k, v, aq, ak, av):
+    """FP8 operands with the scales of given maxima (a_q, a_k scalars; a_v [H, d]): the
+    quantisation of ``quantize_qkv`` with the maxima supplied instead of measured (delayed
+    scaling).  An input above its group's maximum rounds to the code of +-448."""
+    qf, kf, vf = _f32(q), _f32(k), _f32(v)
+    aq, ak = np.float32(aq), np.float32(ak)
+    av = np.asarray(av, dtype=np.float32)
+    out = {"q8": quantize(qf, aq), "k8": quantize(kf, ak), "v8": quantize(vf, av[None, :, :])}
+    out["s_q"] = quant_params(aq)[1]
+    out["s_k"] = quant_params(ak)[1]
+    out["s_v"] = quant_params(av)[1]
+    return out
+
+
 def quantize_qkv(q, k, v):
     """FP8 operands of the variant.
 
     q, k, v: [T, H, d] (bf16 tensors or fp32-valued arrays).  Returns a dict with
     q8, k8, v8 (uint8 codes [T, H, d]), s_q, s_k (fp32 scalars) and s_v (fp32 [H, d]).
     """
-    qf, kf, vf = _f32(q), _f32(k), _f32(v)
-    aq = np.float32(np.max(np.abs(qf))) if qf.size else np.float32(0)
-    ak = np.float32(np.max(np.abs(kf))) if kf.size else np.float32(0)
-    av = (np.max(np.abs(vf), axis=0) if vf.shape[0] else np.zeros(vf.shape[1:])).astype(np.float32)
-    out = {"q8": quantize(qf, aq), "k8": quantize(kf, ak), "v8": quantize(vf, av[None, :, :])}
-    out["s_q"] = quant_params(aq)[1]
-    out["s_k"] = quant_params(ak)[1]
-    out["s_v"] = quant_params(av)[1]
-    return out
+    return quantize_qkv_with(q, k, v, *qkv_amax(q, k, v))
 
 
 def dequantize(codes, s):

@@ -92,6 +92,35 @@ def check_zero_tensor(fp8):
     assert not qz["q8"].any() and qz["s_q"] == 1.0 and np.all(qz["s_v"] == 1.0)
 
 
+def check_maxima_match_torch(fp8):
+    q, k, v, _ = workloads.random_qkv(200, 3, 16, seed=8)
+    aq, ak, av = fp8.qkv_amax(q, k, v)
+    assert aq == q.float().abs().max().item() and ak == k.float().abs().max().item()
+    assert np.array_equal(av, v.float().abs().amax(dim=0).numpy())
+
+
+def check_given_maxima_against_torch(fp8):
+    """Delayed scaling: with maxima above the data's, each code is PyTorch's E4M3 of the fp32
+    product x * (448 / a); with maxima below it, what lies above a saturates to +-448 (codes
+    0x7E / 0xFE) and the rest is PyTorch's E4M3 of the product."""
+    q, k, v, _ = workloads.random_qkv(200, 3, 16, seed=9)
+    aq, ak, av = fp8.qkv_amax(q, k, v)
+    for f in (2.0, 0.5):
+        gq, gk, gv = np.float32(aq * f), np.float32(ak * f), (av * np.float32(f)).astype(np.float32)
+        qz = fp8.quantize_qkv_with(q, k, v, gq, gk, gv)
+        for x, g, codes in ((q, gq, qz["q8"]), (k, gk, qz["k8"]), (v, gv[None, :, :], qz["v8"])):
+            xf = x.float().numpy()
+            mult = (np.float32(448.0) / np.asarray(g, dtype=np.float32)).astype(np.float32)
+            prod = (xf * mult).astype(np.float32)
+            over = np.abs(prod) > 448.0
+            assert over.any() == (f < 1.0)
+            dec = fp8.e4m3_decode(codes)
+            assert np.all(dec[over] == np.sign(prod[over]) * 448.0)
+            assert np.array_equal(dec[~over], _torch_e4m3(prod[~over]).astype(np.float64))
+        assert qz["s_q"] == np.float32(gq) / np.float32(448.0)
+        assert np.array_equal(qz["s_v"], (gv / np.float32(448.0)).astype(np.float32))
+
+
 def _representable(fp8, rng, shape, top):
     """Random E4M3 values times `top` / 448 (a power of two), with the top value present."""
     codes = rng.integers(0, 0x7E, size=shape).astype(np.uint8)
@@ -124,4 +153,4 @@ def check_exact_operands_give_plain_attention(fp8):
     assert not np.array_equal(fp8.e4m3_decode(vz) * (np.max(np.abs(v)) / 448.0), v)
 
 
-ALL_CHECKS = [check_decode_table_matches_torch, check_encode_roundtrips_every_finite_code, check_rounding_matches_torch_in_range, check_ties_go_to_even_mantissa_and_saturate, check_quant_params_closed_forms, check_quantizer_axes_and_error_bound, check_zero_tensor, check_exact_operands_give_plain_attention]
+ALL_CHECKS = [check_decode_table_matches_torch, check_encode_roundtrips_every_finite_code, check_rounding_matches_torch_in_range, check_ties_go_to_even_mantissa_and_saturate, check_quant_params_closed_forms, check_quantizer_axes_and_error_bound, check_zero_tensor, check_exact_operands_give_plain_attention, check_maxima_match_torch, check_given_maxima_against_torch]

@@ -19,7 +19,7 @@ def lib():
 def test_header_declares_the_abi():
     names = pa.header_functions()
     assert "pa_varlen_attn_fwd" in names and "pa_get_error" in names
-    assert len(names) == len(set(names)) == 18
+    assert len(names) == len(set(names)) == 19
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -129,6 +129,15 @@ def test_fp8_host_validation_before_any_cuda_call(lib):
     assert q(*qargs(v8t=24)) == pa.PA_ERR_ALIGN
     assert q(*qargs(scales=8)) == pa.PA_ERR_ALIGN
     assert q(*qargs(total=128 * 65536)) == pa.PA_ERR_SHAPE
+    qd = lib.pa_fp8_quantize_qkv_delayed
+    dargs = lambda **kw: (16, 16, 16, 16, kw.get("batch", 1), kw.get("total", 4), 1, kw.get("d", 128),
+                          kw.get("ain", 4096), kw.get("aout", 8192), 16, 16, 16, 16, None)
+    assert qd(*dargs(d=64)) == pa.PA_ERR_HEAD_DIM
+    assert qd(*dargs(ain=None)) == pa.PA_ERR_NULL
+    assert qd(*dargs(aout=None)) == pa.PA_ERR_NULL
+    assert qd(*dargs(ain=4098)) == pa.PA_ERR_ALIGN
+    assert qd(*dargs(aout=4096 + 8)) == pa.PA_ERR_SHAPE  # overlaps amax_in (4 * (4 + 128) bytes)
+    assert qd(*dargs(batch=0, total=3)) == pa.PA_ERR_SHAPE
     f = lib.pa_varlen_attn_fwd_fp8
     fargs = lambda **kw: (16, 16, kw.get("v8t", 16), kw.get("scales", 16), 16, kw.get("batch", 1), kw.get("total", 4),
                           1, kw.get("d", 128), kw.get("max_seqlen", 4), ctypes.c_float(kw.get("scale", 0.1)),

@@ -215,3 +215,72 @@ def test_fp8_full_size_sampled(pa, config):
     tok, head = workloads.sampled_rows(cfg, per_head=48)
     errs = _compare_rows(p, out, lse, tok.numpy(), head.numpy(), config, qz)
     assert errs["rel_fro"] < 0.05
+
+
+# ---- delayed scaling: scales from given maxima, this call's maxima returned
+
+def _amax_vec(aq, ak, av):
+    a = np.zeros(4 + av.size, dtype=np.float32)
+    a[0], a[1] = aq, ak
+    a[4:] = av.reshape(-1)
+    return a
+
+
+@pytest.mark.parametrize("factor", [2.0, 1.0, 0.5])
+@pytest.mark.parametrize("name", ["ragged", "odd_starts", "empty_ends"])
+def test_delayed_quantiser_bit_exact(pa, name, factor):
+    """Codes and scales from given maxima (above the data's: no saturation; equal: the
+    current-scaling result; below: saturation at +-448) match the oracle bit for bit, and the
+    returned maxima are the data's exactly."""
+    segs, H = PACKS[name]
+    p = workloads.random_pack(segs, H, 128, seed=53)
+    aq, ak, av = fp8.qkv_amax(p["q"], p["k"], p["v"])
+    gq, gk, gv = np.float32(aq * factor), np.float32(ak * factor), (av * np.float32(factor)).astype(np.float32)
+    cu = p["cu_seqlens"].cuda()
+    qz_dev = pa.fp8_quantize_qkv_delayed(p["q"].cuda(), p["k"].cuda(), p["v"].cuda(), cu,
+                                         torch.from_numpy(_amax_vec(gq, gk, gv)).cuda())
+    assert pa.pa_get_error() == pa.PA_OK
+    qz = fp8.quantize_qkv_with(p["q"], p["k"], p["v"], gq, gk, gv)
+    _check_quantiser(pa, p, qz_dev, qz=qz)
+    assert np.array_equal(qz_dev["amax"].cpu().numpy(), _amax_vec(aq, ak, av))
+    if factor == 1.0:  # the same operands as the current-scaling quantiser
+        ref = pa.fp8_quantize_qkv(p["q"].cuda(), p["k"].cuda(), p["v"].cuda(), cu)
+        for key in ("q8", "k8", "scales"):
+            assert torch.equal(ref[key], qz_dev[key]), key
+        # v8t: the segments' keys (the keys between segments are never written)
+        cun = p["cu_seqlens"].numpy()
+        assert np.array_equal(_v8_from_vt(ref["v8t"], cun, H), _v8_from_vt(qz_dev["v8t"], cun, H))
+
+
+def test_delayed_quantiser_two_steps_end_to_end(pa):
+    """A loop of two steps: step 1 quantises with step 0's maxima (returned by step 0's
+    call from all-ones maxima) and the FP8 attention on its operands meets the FP8 bound
+    against the oracle of the dequantised operands."""
+    segs, H = [300, 129, 17, 700], 2
+    p0 = workloads.random_pack(segs, H, 128, seed=61)
+    p1 = workloads.random_pack(segs, H, 128, seed=62)
+    cu = p0["cu_seqlens"].cuda()
+    ones = torch.ones(4 + H * 128, dtype=torch.float32, device="cuda")
+    z0 = pa.fp8_quantize_qkv_delayed(p0["q"].cuda(), p0["k"].cuda(), p0["v"].cuda(), cu, ones)
+    z1 = pa.fp8_quantize_qkv_delayed(p1["q"].cuda(), p1["k"].cuda(), p1["v"].cuda(), cu, z0["amax"])
+    out, lse = pa.varlen_attn_fwd_fp8(z1, cu, p1["max_seqlen"], p1["scale"])
+    assert pa.pa_get_error() == pa.PA_OK
+    a0 = fp8.qkv_amax(p0["q"], p0["k"], p0["v"])
+    assert np.array_equal(z0["amax"].cpu().numpy(), _amax_vec(*a0))
+    qz = fp8.quantize_qkv_with(p1["q"], p1["k"], p1["v"], *a0)
+    _check_quantiser(pa, p1, z1, qz=qz)
+    _compare_full(p1, out, lse, "delayed two steps", qz)
+
+
+def test_delayed_quantiser_empty_pack_zeroes_amax(pa):
+    H = 2
+    amax_in = torch.ones(4 + H * 128, dtype=torch.float32, device="cuda")
+    amax_out = torch.full((4 + H * 128,), 7.0, dtype=torch.float32, device="cuda")
+    e = torch.empty(0, H, 128, dtype=torch.bfloat16, device="cuda")
+    e8 = torch.empty(0, H, 128, dtype=torch.uint8, device="cuda")
+    cu = torch.zeros(1, dtype=torch.int32, device="cuda")
+    vt = torch.empty(H * 128, 0, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(4 + H * 128, dtype=torch.float32, device="cuda")
+    rc = pa.pa_fp8_quantize_qkv_delayed(e, e, e, cu, amax_in, amax_out, e8, e8, vt, sc)
+    assert rc == pa.PA_OK and pa.pa_get_error() == pa.PA_OK
+    assert not amax_out.any()
