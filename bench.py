@@ -392,7 +392,7 @@ class Pack:
             raise pa.PackAttnError(rc, "pa_varlen_attn_fwd")
 
 
-def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5):
+def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5, clocks=None):
     """Per-call time of one pack (L2 flushed before every call) and its kernel alone; the step
     count is the bench's, capped so that the region stays under about `target_s` seconds."""
     pack()
@@ -402,13 +402,16 @@ def measure_pack(pa, pack, flush, stream, args, world, device, target_s=0.5):
     torch.cuda.synchronize()
     est = max(time.time() - t0, 1e-5)
     steps = max(5, min(args.steps, int(target_s / est)))
+    t0 = time.time()
     ms, kms = paired_steps(pa, pack, flush, stream, args.warmup, steps, world, device)
+    t1 = time.time()
     rc = pa.pa_get_error(stream)
     if rc != pa.PA_OK:
         raise pa.PackAttnError(rc, pack.cfg["name"])
     ledger = pa.pa_schedule_stats(stream)  # the tile ledger of the last call
     call_ms = sum(ms) / len(ms)
     return dict(steps=steps, ms_per_call=call_ms, kernel_ms=kms, ledger=ledger,
+                clocks=clocks.summary(t0, t1) if clocks else None,
                 tflops=pack.flops * world / (call_ms * 1e-3) / 1e12,
                 kernel_tflops=pack.flops / (kms * 1e-3) / 1e12,
                 gbs=pack.bytes * world / (call_ms * 1e-3) / 1e9,
@@ -646,7 +649,7 @@ def run_ours(args, world, rank, local):
             if name == args.config:
                 continue
             pk = Pack(pa, workloads.load_config(name), device, stream, seed_offset=7919 * rank)
-            rec = measure_pack(pa, pk, flush, stream, args, world, device)
+            rec = measure_pack(pa, pk, flush, stream, args, world, device, clocks=clocks)
             rec.update(tokens=pk.T, segments=len(pk.segs), heads=pk.H, head_dim=pk.d, valid_flops=pk.flops,
                        unique_bytes=pk.bytes)
             if pk.d == 128 and name in workloads.CONFIG_NAMES and name != "tiny":
@@ -655,7 +658,7 @@ def run_ours(args, world, rank, local):
                 # the same pack with short-segment packing off: every segment its own tiles
                 pa.pa_set_short_packing(False)
                 try:
-                    rec["packing_off"] = measure_pack(pa, pk, flush, stream, args, world, device)
+                    rec["packing_off"] = measure_pack(pa, pk, flush, stream, args, world, device, clocks=clocks)
                 finally:
                     pa.pa_set_short_packing(True)
             per_config[name] = rec
@@ -710,7 +713,8 @@ def run_ours(args, world, rank, local):
              "value": rec["tflops"], "unit": "TFLOP/s", "pct_of_bf16_peak": 100.0 * rec["tflops"] / world / peak_burst,
              "kernel": {"name": head_kernel_name(rec["head_dim"]), "ms": rec["kernel_ms"],
                         "achieved": rec["kernel_tflops"], "frac": rec["kernel_tflops"] / peak_burst,
-                        "peak": peak_burst, "peak_source": f"bf16_tflops ({peak_src}, burst)"}}
+                        "peak": peak_burst, "peak_source": f"bf16_tflops ({peak_src}, burst)"},
+             "clocks": rec.get("clocks")}
         f8 = rec.get("fp8")
         if f8:
             r["fp8_vs_bf16"] = {
@@ -732,7 +736,7 @@ def run_ours(args, world, rank, local):
                 r["packing_off"] = {"ms_per_call": off["ms_per_call"], "value": off["tflops"], "unit": "TFLOP/s",
                                     "gbs": off["gbs"], "kernel_gbs": off["kernel_gbs"],
                                     "tile_utilisation": off["ledger"]["tile_utilisation"],
-                                    "score_tiles": off["ledger"]["score_tiles"]}
+                                    "score_tiles": off["ledger"]["score_tiles"], "clocks": off.get("clocks")}
                 r["packing_speedup"] = off["ms_per_call"] / rec["ms_per_call"]
             short_rec[name] = r
         else:
