@@ -649,6 +649,10 @@ def run_ours(args, world, rank, local):
             if name == args.config:
                 continue
             pk = Pack(pa, workloads.load_config(name), device, stream, seed_offset=7919 * rank)
+            # each pack from the same state as the headline: a short idle gap (the board's power
+            # average recovers), then its own warm-up and a burst region; its clocks are recorded
+            torch.cuda.synchronize()
+            time.sleep(1.0)
             rec = measure_pack(pa, pk, flush, stream, args, world, device, clocks=clocks)
             rec.update(tokens=pk.T, segments=len(pk.segs), heads=pk.H, head_dim=pk.d, valid_flops=pk.flops,
                        unique_bytes=pk.bytes)
@@ -658,6 +662,8 @@ def run_ours(args, world, rank, local):
                 # the same pack with short-segment packing off: every segment its own tiles
                 pa.pa_set_short_packing(False)
                 try:
+                    torch.cuda.synchronize()
+                    time.sleep(1.0)
                     rec["packing_off"] = measure_pack(pa, pk, flush, stream, args, world, device, clocks=clocks)
                 finally:
                     pa.pa_set_short_packing(True)

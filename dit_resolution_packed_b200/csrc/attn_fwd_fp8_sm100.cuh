@@ -602,33 +602,40 @@ __device__ __forceinline__ uint2 quant8(uint4 x, float m) {
   return make_uint2(o[0], o[1]);
 }
 
-// Block (head h, 128-token tile): q8, k8 in q's layout, and v8 transposed to
+// Block (32-token tile, head h): q8, k8 in q's layout, and v8 transposed to
 // [h * 128 + c][key] with segment s's keys starting at 16*ceil(cu[s]/16) + 16*s
 // (for token t of segment s: key t + 16*ceil(cu[s]/16) + 16*s - cu[s]).
 // Also writes the scales: [0] s_q, [1] s_k, [4 + h * 128 + c] s_v.
 // kTrack: the maxima of this call's q, k, v are also accumulated into amax_out (same
 // layout as amax, zeroed by the caller), for the next call's scales (delayed scaling).
+// Small tiles keep the grid many blocks deep, so its last partial wave is short.
+constexpr int kQuantTile = 32;       // tokens per block
+constexpr int kQuantizeThreads = 128;
 template <bool kTrack>
-__global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
+__global__ void __launch_bounds__(kQuantizeThreads) fp8_quantize_kernel(
     const uint4* q, const uint4* k, const uint4* v, const int32_t* cu, int32_t batch, int32_t total, int32_t heads,
     const uint32_t* amax, uint2* q8, uint2* k8, uint8_t* v8t, int64_t vt_keys, float* scales, uint32_t* amax_out) {
-  constexpr int D = 128;
-  __shared__ __align__(16) uint8_t s_t[D][128 + 4];  // [channel][token] of this tile (word-aligned rows)
+  constexpr int D = 128, kT = kQuantTile, NT = kQuantizeThreads;
+  constexpr int kChunks = kT / 16;  // 16-token chunks of the tile
+  static_assert(kT % 16 == 0 && (kT / 4) * (D / 8) == NT, "one 4-token x 8-channel unit per thread");
+  __shared__ __align__(16) uint8_t s_t[D][kT + 4];  // [channel][token] of this tile (word-aligned rows)
   __shared__ float s_mv[D];
-  __shared__ int64_t s_off[128];
-  __shared__ int s_vec[8];  // 16-token chunk goes out as one 16-byte store
+  __shared__ int64_t s_off[kT];
+  __shared__ int s_vec[kChunks];  // 16-token chunk goes out as one 16-byte store
   __shared__ uint32_t s_am[kTrack ? D + 2 : 1];  // this tile's maxima: v per channel, then q, k
-  const int h = blockIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * 128;
+  const int h = blockIdx.y;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kT;
   const float mq = fp8_mult(__ldg(amax)), mk = fp8_mult(__ldg(amax + 1));
-  if (kTrack && threadIdx.x < D + 2) s_am[threadIdx.x] = 0u;
-  if (threadIdx.x < D) {
-    const uint32_t a = __ldg(amax + 4 + h * D + threadIdx.x);
-    s_mv[threadIdx.x] = fp8_mult(a);
-    if (blockIdx.y == 0) scales[4 + h * D + threadIdx.x] = fp8_scale(a);
-  } else if (threadIdx.x - D < 128) {
+  if (kTrack)
+    for (int i = threadIdx.x; i < D + 2; i += NT) s_am[i] = 0u;
+  for (int c = threadIdx.x; c < D; c += NT) {
+    const uint32_t a = __ldg(amax + 4 + h * D + c);
+    s_mv[c] = fp8_mult(a);
+    if (blockIdx.x == 0) scales[4 + h * D + c] = fp8_scale(a);
+  }
+  if (threadIdx.x < kT) {
     // key offset of each token of the tile in the transposed layout
-    const int i = threadIdx.x - D;
+    const int i = threadIdx.x;
     const int64_t t = t0 + i;
     int64_t off = 0;
     if (t < total) {
@@ -652,8 +659,8 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
   // q, k: 8 codes per 16-byte load; v: four tokens of one 8-channel chunk per thread, so
   // that each channel's four codes go to the transposed tile as one 32-bit word
   uint32_t tq = 0u, tk = 0u;  // pairs of bf16 magnitudes (kTrack)
-  for (int i = threadIdx.x; i < 32 * (D / 8); i += kQuantThreads) {
-    const int tg = i >> 4, c8 = i & 15;
+  {
+    const int tg = threadIdx.x >> 4, c8 = threadIdx.x & 15;
     uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // [channel of the chunk]: 4 token bytes
     uint32_t tv[4] = {0u, 0u, 0u, 0u};                   // pairs of bf16 magnitudes of v (kTrack)
 #pragma unroll
@@ -688,9 +695,12 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
     for (int e = 0; e < 8; ++e) *reinterpret_cast<uint32_t*>(&s_t[c8 * 8 + e][tg * 4]) = pk[e];
     if (kTrack) {  // bf16 magnitude bits << 16 are the fp32 bits of the same value
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (tv[e] & 0xFFFFu) atomicMax(&s_am[c8 * 8 + 2 * e], (tv[e] & 0xFFFFu) << 16);
-        if (tv[e] >> 16) atomicMax(&s_am[c8 * 8 + 2 * e + 1], (tv[e] >> 16) << 16);
+      for (int e = 0; e < 4; ++e) {  // lanes l and l + 16 hold the same channels (two token groups)
+        tv[e] = __vmaxu2(tv[e], __shfl_xor_sync(0xffffffffu, tv[e], 16));
+        if ((threadIdx.x & 16) == 0) {
+          if (tv[e] & 0xFFFFu) atomicMax(&s_am[c8 * 8 + 2 * e], (tv[e] & 0xFFFFu) << 16);
+          if (tv[e] >> 16) atomicMax(&s_am[c8 * 8 + 2 * e + 1], (tv[e] >> 16) << 16);
+        }
       }
     }
   }
@@ -706,42 +716,45 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(
       if (fk) atomicMax(&s_am[D + 1], fk);
     }
   }
-  __syncthreads();
-  if (kTrack) {
-    if (threadIdx.x < D) {
-      if (s_am[threadIdx.x]) atomicMax(amax_out + 4 + h * D + threadIdx.x, s_am[threadIdx.x]);
-    } else if (threadIdx.x < D + 2) {
-      if (s_am[threadIdx.x]) atomicMax(amax_out + threadIdx.x - D, s_am[threadIdx.x]);
-    }
-  }
-  // v8^T rows, one warp per channel row: a 16-token chunk goes out as one 16-byte store
-  // when its tokens lie in one segment (equal key offsets: the offset grows at every
-  // segment start) and its first key is 16-byte aligned (decided once per block, the
-  // same for every row); the other tokens as bytes, four consecutive tokens per lane.
-  // Keys are in range for every valid cu_seqlens; the checks keep a malformed one (not
-  // validated here) from writing outside the buffer.
-  if (threadIdx.x < 8) {
+  // v8^T rows: a 16-token chunk goes out as one 16-byte store when its tokens lie in one
+  // segment (equal key offsets: the offset grows at every segment start) and its first key
+  // is 16-byte aligned (decided once per block, the same for every row); the other tokens
+  // as bytes. Keys are in range for every valid cu_seqlens; the checks keep a malformed one
+  // (not validated here) from writing outside the buffer.
+  if (threadIdx.x < kChunks) {
     const int tt0 = threadIdx.x * 16;
     const int64_t t_first = t0 + tt0, key0 = t_first + s_off[tt0];
     s_vec[threadIdx.x] = t_first + 15 < total && s_off[tt0] == s_off[tt0 + 15] && (key0 & 15) == 0 &&
                          key0 >= 0 && key0 + 16 <= vt_keys;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = warp; c < D; c += kQuantThreads / 32) {
-    uint8_t* row = v8t + static_cast<int64_t>(h * D + c) * vt_keys;
-    if (lane < 8 && s_vec[lane]) {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(&s_t[c][lane * 16]);
-      *reinterpret_cast<uint4*>(row + t0 + lane * 16 + s_off[lane * 16]) = make_uint4(src[0], src[1], src[2], src[3]);
+  if (kTrack) {
+    // maxima only grow: a tile whose maximum is not above the value already in amax_out
+    // (read from L2) skips its atomic, so the two whole-tensor words are not hit by every block
+    for (int i = threadIdx.x; i < D + 2; i += NT) {
+      uint32_t* dst = i < D ? amax_out + 4 + h * D + i : amax_out + i - D;
+      if (s_am[i] > __ldcg(dst)) atomicMax(dst, s_am[i]);
     }
-    if (!s_vec[lane >> 2]) {
+  }
+  // (channel row, chunk) pairs, chunk fastest: 16-byte stores
+  for (int j = threadIdx.x; j < D * kChunks; j += NT) {
+    const int c = j / kChunks, ch = j % kChunks;
+    if (!s_vec[ch]) continue;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&s_t[c][ch * 16]);
+    uint8_t* row = v8t + static_cast<int64_t>(h * D + c) * vt_keys;
+    *reinterpret_cast<uint4*>(row + t0 + ch * 16 + s_off[ch * 16]) = make_uint4(src[0], src[1], src[2], src[3]);
+  }
+  // (channel row, 4-token group) pairs of the other chunks: bytes
+  for (int j = threadIdx.x; j < D * (kT / 4); j += NT) {
+    const int c = j / (kT / 4), g = j % (kT / 4);
+    if (s_vec[g >> 2]) continue;
+    uint8_t* row = v8t + static_cast<int64_t>(h * D + c) * vt_keys;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tt = lane * 4 + e;
-        const int64_t t = t0 + tt;
-        const int64_t key = t + s_off[tt];
-        if (t < total && key >= 0 && key < vt_keys) row[key] = s_t[c][tt];
-      }
+    for (int e = 0; e < 4; ++e) {
+      const int tt = g * 4 + e;
+      const int64_t t = t0 + tt;
+      const int64_t key = t + s_off[tt];
+      if (t < total && key >= 0 && key < vt_keys) row[key] = s_t[c][tt];
     }
   }
 }

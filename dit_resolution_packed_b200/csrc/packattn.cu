@@ -882,8 +882,8 @@ int fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q8, 16) || !aligned(k8, 16) ||
       !aligned(v8t, 16) || !aligned(scales, 16) || !aligned(cu_seqlens, 4))
     return PA_ERR_ALIGN;
-  const int64_t tiles = (static_cast<int64_t>(total_tokens) + 127) / 128;
-  if (tiles > 65535 || heads > 65535 || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24) ||
+  const int64_t tiles = (static_cast<int64_t>(total_tokens) + pa::kQuantTile - 1) / pa::kQuantTile;
+  if (heads > 65535 || static_cast<int64_t>(heads) * head_dim >= (int64_t(1) << 24) ||
       fp8_vt_keys(batch, total_tokens) >= (int64_t(1) << 32))
     return PA_ERR_SHAPE;
   int dev = -1, d2 = -1;
@@ -898,11 +898,11 @@ int fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_
   std::lock_guard<std::mutex> lock(g_mu);
   if (cudaSetDevice(dev) != cudaSuccess) return PA_ERR_CUDA;
   if ((rc = ensure_device(dev)) != PA_OK) return rc;
-  const dim3 qgrid(heads, static_cast<unsigned>(tiles));
+  const dim3 qgrid(static_cast<unsigned>(tiles), heads);
   const int64_t vt_keys = fp8_vt_keys(batch, total_tokens);
   if (delayed) {
     if (cudaMemsetAsync(amax_out, 0, amax_bytes, stream) != cudaSuccess) return PA_ERR_CUDA;
-    pa::fp8_quantize_kernel<true><<<qgrid, pa::kQuantThreads, 0, stream>>>(
+    pa::fp8_quantize_kernel<true><<<qgrid, pa::kQuantizeThreads, 0, stream>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, batch,
         total_tokens, heads, reinterpret_cast<const uint32_t*>(amax_in), static_cast<uint2*>(q8),
         static_cast<uint2*>(k8), static_cast<uint8_t*>(v8t), vt_keys, scales, reinterpret_cast<uint32_t*>(amax_out));
@@ -921,7 +921,7 @@ int fp8_quantize(const void* q, const void* k, const void* v, const int32_t* cu_
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), total_tokens, nch8,
       amax);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  pa::fp8_quantize_kernel<false><<<qgrid, pa::kQuantThreads, 0, stream>>>(
+  pa::fp8_quantize_kernel<false><<<qgrid, pa::kQuantizeThreads, 0, stream>>>(
       static_cast<const uint4*>(q), static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, batch,
       total_tokens, heads, amax, static_cast<uint2*>(q8), static_cast<uint2*>(k8), static_cast<uint8_t*>(v8t),
       vt_keys, scales, nullptr);

@@ -120,15 +120,15 @@ def test_fp8_host_validation_before_any_cuda_call(lib):
     assert pa.pa_fp8_vt_keys(1, 16) == 32 and pa.pa_fp8_vt_keys(0, 0) == 0
     assert pa.pa_fp8_vt_keys(-1, 4) == -1
     q = lib.pa_fp8_quantize_qkv
-    qargs = lambda **kw: (kw.get("q", 16), 16, 16, kw.get("cu", 16), kw.get("batch", 1), kw.get("total", 4), 1,
-                          kw.get("d", 128), 16, 16, kw.get("v8t", 16), kw.get("scales", 16), None)
+    qargs = lambda **kw: (kw.get("q", 16), 16, 16, kw.get("cu", 16), kw.get("batch", 1), kw.get("total", 4),
+                          kw.get("heads", 1), kw.get("d", 128), 16, 16, kw.get("v8t", 16), kw.get("scales", 16), None)
     assert q(*qargs(d=64)) == pa.PA_ERR_HEAD_DIM
     assert q(*qargs(batch=0, total=3)) == pa.PA_ERR_SHAPE
     assert q(*qargs(batch=0, total=0)) == pa.PA_OK
     assert q(*qargs(q=None)) == pa.PA_ERR_NULL
     assert q(*qargs(v8t=24)) == pa.PA_ERR_ALIGN
     assert q(*qargs(scales=8)) == pa.PA_ERR_ALIGN
-    assert q(*qargs(total=128 * 65536)) == pa.PA_ERR_SHAPE
+    assert q(*qargs(heads=65536)) == pa.PA_ERR_SHAPE
     qd = lib.pa_fp8_quantize_qkv_delayed
     dargs = lambda **kw: (16, 16, 16, 16, kw.get("batch", 1), kw.get("total", 4), 1, kw.get("d", 128),
                           kw.get("ain", 4096), kw.get("aout", 8192), 16, 16, 16, 16, None)
